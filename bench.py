@@ -1,0 +1,381 @@
+"""Benchmark of the absorbed MLA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload v3] [--num-splits P]
+
+One step = one pass of the whole hot path over one batch: mla_absorb_q
+(q_nope . W_UK, packed with q_rope) then mla_decode (split-KV decode over the
+paged latent cache, then the LSE merge of cut sequences).  Inputs are seeded
+synthetic tensors of the DeepSeek-V3 decode shape (B=64, H=128, L=4096, bf16
+paged cache in 64-token blocks under a random block permutation), resident in
+HBM before timing.  The cache (302 MB) is larger than L2 (126 MB), so no L2
+flush is needed between steps.
+
+value = algorithmic bytes of one step (cache rows of every token once, the
+query, the output and lse, W_UK and the absorption inputs/outputs) divided by
+the device time per step (CUDA events, max over ranks), in GB/s.
+
+Multi-GPU: the decode of independent batches does not exchange anything, so
+N ranks run N independent replicas (weak scaling); the only collective is
+the max-over-ranks of the timings.
+
+--impl reference times the FP64 CPU oracle on a bounded sample of the same
+workload (the reference arm of this method is the oracle).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mla_latent_kv_25_b200 import inputs, layout  # noqa: E402
+
+METRIC = "MLA decode: cache GB/s and TFLOP/s vs roofline at DeepSeek-V3 shapes, 1 B200"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="v3", choices=list(inputs.CONFIGS))
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources: a stored ncu traffic figure is only reported
+    while the kernels it was taken from are unchanged."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_latent_kv_25_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode())
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload: str):
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu
+    summary (profiles/traffic_<workload>.txt: 'kernel_hash <h>' and
+    'dram_bytes_per_launch <n>' lines), or None when absent or stale."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{workload}.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 2:
+            kv[parts[0]] = parts[1]
+    if kv.get("kernel_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def step_bytes_flops(w):
+    dec_b = layout.decode_algorithmic_bytes(w.total_tokens, w.B, w.H, w.cache_dtype,
+                                            num_blocks_read=int(((w.seq_lens + 63) // 64).sum()))
+    abs_b = layout.absorb_algorithmic_bytes(w.B, w.H)
+    dec_f = layout.decode_flops(w.total_tokens, w.H)
+    abs_f = layout.absorb_flops(w.B, w.H)
+    return dec_b, abs_b, dec_f, abs_f
+
+
+def run_ours(args, world, rank, local):
+    from mla_latent_kv_25_b200 import binding
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    w = inputs.make(args.workload, seed=inputs.CONFIGS[args.workload]["seed"] + 1000 * rank)
+    d = binding.to_device(w, dev)
+    B, H = w.B, w.H
+    stream = torch.cuda.current_stream(dev)
+    q = torch.empty((B, H, 576), dtype=torch.bfloat16, device=dev)
+    q_rope = w.q[:, :, 512:].contiguous().to(dev)
+    out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    ws = binding.alloc_workspace(B, H, args.num_splits, device=dev)
+    dec_b, abs_b, dec_f, abs_f = step_bytes_flops(w)
+
+    def step():
+        binding.mla_absorb_q(d["q_nope"], d["w_uk"], q_rope, q, stream=stream)
+        binding.mla_decode(q, d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale, out,
+                           lse, ws, k_rope=d["k_rope"], block_scale=d["block_scale"],
+                           num_splits=args.num_splits, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if binding.mla_get_device_error(ws, stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    # device-timed region: K steps, decode calls bracketed by events as well
+    K = args.steps
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(K):
+        binding.mla_absorb_q(d["q_nope"], d["w_uk"], q_rope, q, stream=stream)
+        ev_dec[i][0].record(stream)
+        binding.mla_decode(q, d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale, out,
+                           lse, ws, k_rope=d["k_rope"], block_scale=d["block_scale"],
+                           num_splits=args.num_splits, stream=stream)
+        ev_dec[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = t0.elapsed_time(t1)
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
+
+    # end to end through the public API with host buffers: per step copy the
+    # new queries (q_nope, q_rope) host->device, run the step, copy out/lse back
+    h_qn = w.q_nope.pin_memory()
+    h_qr = w.q[:, :, 512:].contiguous().pin_memory()
+    h_out = torch.empty((B, H, 512), dtype=torch.bfloat16).pin_memory()
+    h_lse = torch.empty((B, H), dtype=torch.float32).pin_memory()
+    K2 = max(1, K // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K2):
+        d["q_nope"].copy_(h_qn, non_blocking=True)
+        q_rope.copy_(h_qr, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / K2
+    clk = clocks.stop()
+    if binding.mla_get_device_error(ws, stream) != 0:
+        raise RuntimeError("device error during timing")
+
+    step_ms = ms / K
+    if world > 1:
+        t = torch.tensor([step_ms, dec_ms, e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms, dec_ms, e2e_ms = (float(x) for x in t.tolist())
+
+    res = None
+    if rank == 0:
+        peaks, src = load_peaks()
+        hbm = float(peaks["hbm_gbs"])
+        tens = float(peaks["bf16_tflops"])
+        step_bytes = dec_b + abs_b
+        value = step_bytes * world / (step_ms * 1e-3) / 1e9
+        achieved = dec_b / (dec_ms * 1e-3) / 1e9
+        dec_tflops = dec_f / (dec_ms * 1e-3) / 1e12
+        t_hbm = dec_b / (hbm * 1e9)
+        t_tc = dec_f / (tens * 1e12)
+        bound = "hbm" if t_hbm >= t_tc else "tensor"
+        traffic = stored_traffic(args.workload)
+        if bound == "hbm":
+            roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved / hbm, 4)}
+        else:
+            roof = {"bound": "tensor", "achieved": round(dec_tflops, 1), "peak": tens,
+                    "unit": "TFLOP/s", "frac": round(dec_tflops / tens, 4)}
+        roof["traffic"] = traffic
+        roof["algorithmic_bytes"] = dec_b
+        roof["kernel"] = "mla_decode (decode kernel + merge kernel)"
+        roof["ms_per_launch"] = round(dec_ms, 5)
+        roof["roofline_ms"] = round(max(t_hbm, t_tc) * 1e3, 5)
+        roof["peak_source"] = f"{src} ({'MEASURED_PEAKS.json' if src == 'measured' else 'fallback'})"
+        res = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": max(3, args.warmup),
+            "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if w.cache_dtype == "bf16" else "fp8-e4m3 cache, bf16 mma",
+            "data": "synthetic (seeded; DeepSeek-V3 decode shape, random-permuted paged cache)",
+            "config": {"workload": args.workload, "description": inputs.DESCRIPTIONS[args.workload],
+                       "B": B, "H": H, "tokens": w.total_tokens, "cache": w.cache_dtype,
+                       "num_splits": args.num_splits,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (cache %.0f MB > 126 MB); no flush"
+                             % (w.cache.numel() * w.cache.element_size() / 1e6)},
+            "tflops": round((dec_f + abs_f) * world / (step_ms * 1e-3) / 1e12, 2),
+            "decode_tflops": round(dec_tflops, 2),
+            "roofline": roof,
+            "e2e": {"value": round(step_bytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "ms_per_step": round(e2e_ms, 5),
+                    "h2d_bytes_per_step": int(h_qn.numel() * 2 + h_qr.numel() * 2),
+                    "d2h_bytes_per_step": int(h_out.numel() * 2 + h_lse.numel() * 4)},
+            "gpu_launches": 3 * K,
+            "clocks": clk,
+        }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return res, w
+
+
+def oracle_sample_rate(w, seconds: float, n_seq_max=None):
+    """Time the oracle on whole sequences of the workload until ~``seconds``
+    of work; returns (GB/s of algorithmic bytes, threads, description)."""
+    import oracle
+    cores = oracle.max_threads()
+    done_tokens = 0
+    rows = 0
+    t_total = 0.0
+    b = 0
+    while b < w.B and t_total < seconds and (n_seq_max is None or b < n_seq_max):
+        units = np.stack([np.full(w.H, b), np.arange(w.H), np.zeros(w.H), -np.ones(w.H)], 1)
+        t = time.perf_counter()
+        oracle.decode_units(q=w.q, cache=w.cache, block_table=w.block_table, seq_lens=w.seq_lens,
+                            num_blocks=w.num_blocks, softmax_scale=w.softmax_scale,
+                            units=units.astype(np.int32), cache_kind=w.cache_dtype,
+                            k_rope=w.k_rope, block_scale=w.block_scale)
+        t_total += time.perf_counter() - t
+        done_tokens += int(w.seq_lens[b])
+        rows += w.H
+        b += 1
+    nb = int((done_tokens + 63) // 64)
+    by = layout.decode_algorithmic_bytes(done_tokens, b, w.H, w.cache_dtype, nb)
+    desc = f"{b} of {w.B} sequences x {w.H} heads ({done_tokens} tokens) of workload {w.name}"
+    return by / t_total / 1e9, cores, desc, t_total
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = inputs.make(args.workload)
+    dec_b, abs_b, _, _ = step_bytes_flops(w)
+    vals = []
+    K = max(1, min(args.steps, 3))
+    desc, cores = "", 1
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample_rate(w, 0.0, n_seq_max=1)
+    per = max(1.0, args.cpu_seconds / K)
+    for _ in range(K):
+        v, cores, desc, _t = oracle_sample_rate(w, per)
+        vals.append(v)
+    v = float(np.median(vals))
+    ms = (dec_b + abs_b) / (v * 1e9) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": args.workload, "description": inputs.DESCRIPTIONS[args.workload]},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": desc + " per step"},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    res, w = run_ours(args, world, rank, local)
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            v, cores, desc, t = oracle_sample_rate(w, args.cpu_seconds)
+            res["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores,
+                                   "kind": "oracle", "sample": desc + f", {t:.1f} s"}
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+/*
+ * mla.h - C ABI of libmla.so: absorbed Multi-Head Latent Attention decode over
+ * a paged latent KV cache, hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * The method ("Multi-Head Latent Attention: Scaling LLM Serving Throughput via
+ * Low-Rank KV Compression", priorstack.com, sections "Empirical Gains" and
+ * "Frequently Asked Questions"): every cached token keeps one shared row
+ * [c_kv (d_c = 512) | k_rope (d_h^R = 64)]; the key up-projection W_UK is
+ * absorbed into the query and W_UV into the output projection, so the decode
+ * step attends directly over the latent rows:
+ *
+ *     q_abs[b,h,:] = q_nope[b,h,:] . W_UK[h]                        (512)
+ *     s[b,h,t]     = scale * (q_abs[b,h,:] . c_kv[t] + q_rope[b,h,:] . k_rope[t])
+ *     out[b,h,:]   = sum_t softmax_t(s[b,h,:]) c_kv[t]               (512)
+ *     lse[b,h]     = log sum_t exp(s[b,h,t])                         (natural log)
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise, owned by
+ *     the caller.  The library allocates no memory and never synchronises the
+ *     stream (except mla_get_device_error, which says so).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All work is enqueued on it in order.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns an error status and launches nothing.
+ *   - A launch failure returns MLA_ERR_CUDA (cudaGetLastError is consumed).
+ *   - Fixed dimensions: d_c = 512, d_h^R = 64, row = 576, 64 tokens per cache
+ *     block, 128-wide content query (d_h) for absorption.  H must be a
+ *     multiple of 16 in [16, 128].
+ *   - bf16 = IEEE binary32 upper half; fp8 = OCP E4M3 (bias 7, max 448, NaN
+ *     S.1111.111, no infinities).  Outputs are rounded to nearest even.
+ *   - Thread safety: stateless; concurrent calls on different streams are safe
+ *     provided they use different output and workspace buffers.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,         /* null pointer, bad size or alignment */
+    MLA_ERR_UNSUPPORTED = 2,         /* valid request this build does not handle */
+    MLA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < mla_decode_workspace_bytes(...) */
+    MLA_ERR_CUDA = 4,                /* a CUDA runtime/driver call or launch failed */
+    MLA_ERR_DEVICE = 5               /* device-side error bits were set (mla_get_device_error) */
+} mla_status_t;
+
+typedef enum {
+    MLA_CACHE_BF16 = 0,     /* cache: bf16 [num_blocks, 64, 576] rows [c_kv | k_rope] */
+    MLA_CACHE_FP8_E4M3 = 1  /* cache: u8 E4M3 [num_blocks, 64, 512] codes of c_kv / block_scale,
+                               k_rope: bf16 [num_blocks, 64, 64], block_scale: f32 [num_blocks] */
+} mla_cache_dtype_t;
+
+/* Device-side error bits (read with mla_get_device_error). */
+#define MLA_DEVERR_BAD_BLOCK   0x1u  /* a block_table entry needed by seq_lens is < 0 or >= num_blocks */
+#define MLA_DEVERR_SEQ_TOO_LONG 0x2u /* seq_lens[b] > 64 * max_blocks_per_seq or < 0 */
+#define MLA_DEVERR_TIMEOUT     0x4u  /* a bounded wait inside a kernel gave up; the kernel exited */
+
+/*
+ * mla_absorb_q - fold the key up-projection into the query ("Empirical Gains":
+ * W^UK is absorbed into the query projection):
+ *     q_out[(b*H + h)*ldq + c]       = sum_{d<128} q_nope[b,h,d] * w_uk[h,d,c],  c < 512
+ *     q_out[(b*H + h)*ldq + 512 + r] = q_rope[b,h,r],  r < 64   (only if q_rope != NULL)
+ * q_nope: bf16 [B,H,128]; w_uk: bf16 [H,128,512]; q_rope: bf16 [B,H,64] or NULL;
+ * q_out: bf16 rows of stride ldq elements (ldq >= 512, >= 576 if q_rope != NULL,
+ * a multiple of 8; 576 builds the packed [B,H,576] query mla_decode reads).
+ * fp32 accumulation, one bf16 rounding.  B >= 1.  All pointers 16-byte aligned.
+ */
+mla_status_t mla_absorb_q(const void *q_nope, const void *w_uk, const void *q_rope,
+                          void *q_out, int ldq, int B, int H, void *stream);
+
+/*
+ * mla_decode_workspace_bytes - bytes of device workspace mla_decode needs for
+ * H heads and `num_splits` split-KV partitions (0 = the automatic count the
+ * current device would use).  The workspace holds the device error word and
+ * the fp32 partial results of sequences that are cut across partitions.
+ * Returns 0 on invalid arguments.
+ */
+size_t mla_decode_workspace_bytes(int B, int H, int num_splits);
+
+/*
+ * mla_decode - the decode-step attention over the paged latent cache
+ * ("Empirical Gains": the cache holds only c^KV and the decoupled RoPE key;
+ * "The Memory Wall": the whole cache is streamed from HBM every step).
+ *
+ * q:           bf16 [B,H,576] = [q_abs | q_rope] per (b,h) (from mla_absorb_q).
+ * cache_dtype: MLA_CACHE_BF16 or MLA_CACHE_FP8_E4M3 (see the enum).
+ * cache:       bf16 [num_blocks,64,576] or u8 [num_blocks,64,512].
+ * k_rope:      fp8 cache only: bf16 [num_blocks,64,64]; must be NULL for bf16.
+ * block_scale: fp8 cache only: f32 [num_blocks], c_kv = e4m3(code) * scale;
+ *              must be NULL for bf16.
+ * block_table: int32 [B, max_blocks_per_seq]; logical block j of sequence b is
+ *              physical block block_table[b*max_blocks_per_seq + j].  Entries
+ *              at j >= ceil(seq_lens[b]/64) are never read (pad with -1).
+ * seq_lens:    int32 [B] on the device; 0 <= seq_lens[b] <= 64*max_blocks_per_seq.
+ * softmax_scale: multiplies the whole score (both terms) before the softmax.
+ * out:         bf16 [B,H,512], the softmax-weighted sum of c_kv per head.
+ * lse:         f32 [B,H], natural log of sum_t exp(score); a sequence of
+ *              length 0 gives out = 0 and lse = -inf.
+ * workspace:   device buffer of >= mla_decode_workspace_bytes(B,H,num_splits)
+ *              bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE; the
+ *              library keeps its error word zero except when it records an
+ *              error.  One workspace must not be shared by calls that may run
+ *              at the same time.
+ * num_splits:  number of split-KV partitions (0 = automatic).  Results do not
+ *              depend on the physical block placement; they may differ in the
+ *              last bits between different num_splits.
+ *
+ * Preconditions checked on the host: non-null pointers, B >= 1, H in
+ * {16,32,...,128}, num_blocks >= 1, max_blocks_per_seq >= 1, 16-byte
+ * alignment, the fp8-only pointers present exactly for the fp8 cache.
+ * Checked on the device (recorded as error bits, the offending rows are
+ * skipped): block ids in range, seq_lens in range.  Every internal wait is
+ * bounded; on expiry the kernel records MLA_DEVERR_TIMEOUT and exits cleanly.
+ */
+mla_status_t mla_decode(const void *q, mla_cache_dtype_t cache_dtype, const void *cache,
+                        const void *k_rope, const float *block_scale,
+                        const int32_t *block_table, const int32_t *seq_lens, int B, int H,
+                        int num_blocks, int max_blocks_per_seq, float softmax_scale,
+                        void *out, float *lse, void *workspace, size_t workspace_bytes,
+                        int num_splits, void *stream);
+
+/*
+ * mla_combine - log-sum-exp merge of S split-KV partial results (the
+ * flash-decoding merge that makes split-KV equal the unsplit softmax):
+ *     M = max_i lse_part[r,i];  lse[r] = M + log sum_i exp(lse_part[r,i] - M)
+ *     out[r,:] = sum_i exp(lse_part[r,i] - lse[r]) * o_part[r,i,:]
+ * with r = b*H + h.  o_part: f32 [B,H,S,512] (each piece already normalised by
+ * its own softmax sum); lse_part: f32 [B,H,S] (-inf marks an empty piece);
+ * out: bf16 [B,H,512]; lse: f32 [B,H].  Rows whose pieces are all -inf give
+ * out = 0, lse = -inf.  S >= 1.
+ */
+mla_status_t mla_combine(const float *o_part, const float *lse_part, int B, int H, int S,
+                         void *out, float *lse, void *stream);
+
+/*
+ * mla_get_device_error - wait for `stream`, read the MLA_DEVERR_* bits that
+ * kernels using `workspace` recorded, and reset them to zero.  *err_bits
+ * receives the bits.  Returns MLA_OK, or MLA_ERR_CUDA if the stream or copy
+ * failed.  This is the only entry point that synchronises.
+ */
+mla_status_t mla_get_device_error(void *workspace, void *stream, uint32_t *err_bits);
+
+/* mla_status_string - a static, human-readable name for a status code. */
+const char *mla_status_string(mla_status_t status);
+
+/* mla_num_sms - streaming multiprocessors of the current device (0 on error). */
+int mla_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -1,0 +1,170 @@
+// C ABI of libmla.so (declared in include/mla.h): host-side validation,
+// workspace layout, choice of the split-KV engine count, and the launches.
+#include <math.h>
+#include <mutex>
+
+#include "../../include/mla.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+using namespace mla;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static std::mutex mu;
+  static int cache[64] = {0};
+  std::lock_guard<std::mutex> g(mu);
+  if (dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Engines of the split-KV partition: one per pair of SMs by default.
+int resolve_engines(int num_splits) {
+  if (num_splits > 0) return num_splits;
+  int sms = device_sms();
+  return sms >= 2 ? sms / 2 : 1;
+}
+
+constexpr int kMaxSplits = 4096;
+constexpr int kMaxBatch = 1 << 20;
+constexpr long long kDefaultSpin = 4000000000LL;  // ~2 s of SM clock
+
+bool valid_heads(int H) { return H >= 16 && H <= kMaxHeads && H % 16 == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE_TOO_SMALL: return "MLA_ERR_WORKSPACE_TOO_SMALL";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE: return "MLA_ERR_DEVICE";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+int mla_num_sms(void) { return device_sms(); }
+
+size_t mla_decode_workspace_bytes(int B, int H, int num_splits) {
+  if (B < 1 || B > kMaxBatch || !valid_heads(H) || num_splits < 0 || num_splits > kMaxSplits)
+    return 0;
+  int P = resolve_engines(num_splits);
+  if (P < 1) return 0;
+  return ws_layout(B, H, P).total;
+}
+
+mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, const void* q_rope, void* q_out,
+                          int ldq, int B, int H, void* stream) {
+  if (!q_nope || !w_uk || !q_out) return MLA_ERR_INVALID_ARG;
+  if (B < 1 || B > kMaxBatch || !valid_heads(H)) return MLA_ERR_INVALID_ARG;
+  if (ldq < (q_rope ? kRow : kDc) || ldq % 8 != 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || !aligned16(w_uk) || !aligned16(q_out) || (q_rope && !aligned16(q_rope)))
+    return MLA_ERR_INVALID_ARG;
+  cudaError_t e = launch_absorb_q(static_cast<const __nv_bfloat16*>(q_nope),
+                                  static_cast<const __nv_bfloat16*>(w_uk),
+                                  static_cast<const __nv_bfloat16*>(q_rope),
+                                  static_cast<__nv_bfloat16*>(q_out), ldq, B, H,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void* cache,
+                        const void* k_rope, const float* block_scale, const int32_t* block_table,
+                        const int32_t* seq_lens, int B, int H, int num_blocks,
+                        int max_blocks_per_seq, float softmax_scale, void* out, float* lse,
+                        void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
+  if (!q || !cache || !block_table || !seq_lens || !out || !lse || !workspace)
+    return MLA_ERR_INVALID_ARG;
+  if (B < 1 || B > kMaxBatch || !valid_heads(H)) return MLA_ERR_INVALID_ARG;
+  if (num_blocks < 1 || max_blocks_per_seq < 1 || max_blocks_per_seq > (1 << 24))
+    return MLA_ERR_INVALID_ARG;
+  if (num_splits < 0 || num_splits > kMaxSplits) return MLA_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale) || isinf(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  const bool fp8 = (cache_dtype == MLA_CACHE_FP8_E4M3);
+  if (cache_dtype != MLA_CACHE_BF16 && !fp8) return MLA_ERR_INVALID_ARG;
+  if (fp8 != (k_rope != nullptr) || fp8 != (block_scale != nullptr)) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(cache) || !aligned16(out) || (k_rope && !aligned16(k_rope)) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0 ||
+      (block_scale && (reinterpret_cast<uintptr_t>(block_scale) & 3u) != 0))
+    return MLA_ERR_INVALID_ARG;
+  const int P = resolve_engines(num_splits);
+  if (P < 1) return MLA_ERR_CUDA;
+  const WsLayout ws = ws_layout(B, H, P);
+  if (workspace_bytes < ws.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.cache = cache;
+  p.k_rope = static_cast<const __nv_bfloat16*>(k_rope);
+  p.block_scale = block_scale;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.B = B;
+  p.H = H;
+  p.num_blocks = num_blocks;
+  p.max_blocks = max_blocks_per_seq;
+  p.softmax_scale = softmax_scale;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.err = reinterpret_cast<uint32_t*>(wsb);
+  p.seq_info = reinterpret_cast<int4*>(wsb + ws.seq_info);
+  p.lse_part = reinterpret_cast<float*>(wsb + ws.lse_part);
+  p.o_part = reinterpret_cast<float*>(wsb + ws.o_part);
+  p.P = P;
+  p.spin_limit = kDefaultSpin;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  cudaError_t e = launch_decode_simt(p, fp8, st);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  e = launch_merge_pieces(seq_lens, B, max_blocks_per_seq, H, p.seq_info, p.lse_part, p.o_part,
+                          p.out, p.lse, p.err, st);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_combine(const float* o_part, const float* lse_part, int B, int H, int S,
+                         void* out, float* lse, void* stream) {
+  if (!o_part || !lse_part || !out || !lse) return MLA_ERR_INVALID_ARG;
+  if (B < 1 || B > kMaxBatch || H < 1 || H > kMaxHeads || S < 1 || S > (1 << 20))
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o_part) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse_part) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return MLA_ERR_INVALID_ARG;
+  cudaError_t e = launch_combine(o_part, lse_part, B, H, S, static_cast<__nv_bfloat16*>(out), lse,
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_get_device_error(void* workspace, void* stream, uint32_t* err_bits) {
+  if (!workspace || !err_bits) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  *err_bits = v;
+  if (v != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof v, st) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
+}  // extern "C"

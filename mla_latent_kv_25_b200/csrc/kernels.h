@@ -1,0 +1,44 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mla {
+
+struct DecodeParams {
+  const __nv_bfloat16* q;          // [B,H,576]
+  const void* cache;               // bf16 [NB,64,576] | u8 [NB,64,512]
+  const __nv_bfloat16* k_rope;     // fp8 cache: [NB,64,64]
+  const float* block_scale;        // fp8 cache: [NB]
+  const int32_t* block_table;      // [B,max_blocks]
+  const int32_t* seq_lens;         // [B]
+  int B, H, num_blocks, max_blocks;
+  float softmax_scale;
+  __nv_bfloat16* out;              // [B,H,512]
+  float* lse;                      // [B,H]
+  uint32_t* err;                   // workspace error word
+  int4* seq_info;                  // [B]
+  float* lse_part;                 // [2P,H]
+  float* o_part;                   // [2P,H,512]
+  int P;                           // number of split-KV engines
+  long long spin_limit;            // bounded-wait limit (clock64 cycles)
+};
+
+// CUDA-core scaffold decode (any H multiple of 16); fp8: cache is E4M3.
+cudaError_t launch_decode_simt(const DecodeParams& p, bool fp8, cudaStream_t stream);
+
+cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H,
+                                const int4* seq_info, const float* lse_part, const float* o_part,
+                                __nv_bfloat16* out, float* lse, uint32_t* err,
+                                cudaStream_t stream);
+
+cudaError_t launch_combine(const float* o_part, const float* lse_part, int B, int H, int S,
+                           __nv_bfloat16* out, float* lse, cudaStream_t stream);
+
+cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* w_uk,
+                            const __nv_bfloat16* q_rope, __nv_bfloat16* q_out, int ldq, int B,
+                            int H, cudaStream_t stream);
+
+}  // namespace mla

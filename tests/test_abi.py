@@ -1,0 +1,94 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point include/mla.h declares, and rejects invalid arguments on the host
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_latent_kv_25_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "mla.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("mla_absorb_q", "mla_decode", "mla_combine", "mla_decode_workspace_bytes",
+              "mla_get_device_error", "mla_status_string"):
+        assert n in names
+    assert set(names) == set(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = binding.load()
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+        assert isinstance(getattr(lib, n), ctypes._CFuncPtr)
+
+
+def test_status_strings():
+    for code, name in binding.STATUS.items():
+        assert binding.mla_status_string(code) == name
+
+
+def test_workspace_size_and_validation_without_device():
+    lib = binding.load()
+    # explicit split count: no device query needed
+    n1 = lib.mla_decode_workspace_bytes(64, 128, 74)
+    n2 = lib.mla_decode_workspace_bytes(64, 128, 148)
+    assert n1 > 0 and n2 > n1 and n1 % 256 == 0
+    # room for 2 fp32 pieces (512 + lse) per engine and head
+    assert n1 >= 2 * 74 * 128 * 513 * 4
+    assert lib.mla_decode_workspace_bytes(64, 100, 74) == 0     # H not a multiple of 16
+    assert lib.mla_decode_workspace_bytes(64, 256, 74) == 0     # H > 128
+    assert lib.mla_decode_workspace_bytes(0, 128, 74) == 0
+    assert lib.mla_decode_workspace_bytes(1, 128, -1) == 0
+
+
+@pytest.mark.parametrize("case", ["null_q", "bad_heads", "bad_batch", "fp8_missing_rope",
+                                  "bf16_with_scale", "bad_scale", "misaligned"])
+def test_decode_rejects_invalid_arguments_on_host(case):
+    lib = binding.load()
+    P = ctypes.c_void_p
+    good = P(4096)
+    args = dict(q=good, kind=0, cache=good, k_rope=None, scale=None, table=good, lens=good,
+                B=4, H=128, NB=10, maxb=4, sm=0.07, out=good, lse=good, ws=P(256 * 64),
+                wsb=1 << 30, splits=2, stream=None)
+    if case == "null_q":
+        args["q"] = None
+    elif case == "bad_heads":
+        args["H"] = 40
+    elif case == "bad_batch":
+        args["B"] = 0
+    elif case == "fp8_missing_rope":
+        args["kind"] = 1
+        args["scale"] = good
+    elif case == "bf16_with_scale":
+        args["scale"] = good
+    elif case == "bad_scale":
+        args["sm"] = float("nan")
+    elif case == "misaligned":
+        args["cache"] = P(4096 + 2)
+    st = lib.mla_decode(args["q"], args["kind"], args["cache"], args["k_rope"], args["scale"],
+                        args["table"], args["lens"], args["B"], args["H"], args["NB"], args["maxb"],
+                        args["sm"], args["out"], args["lse"], args["ws"], args["wsb"],
+                        args["splits"], args["stream"])
+    assert st == 1, binding.STATUS.get(st, st)
+
+
+def test_absorb_and_combine_reject_invalid_arguments_on_host():
+    lib = binding.load()
+    P = ctypes.c_void_p
+    g = P(4096)
+    assert lib.mla_absorb_q(None, g, None, g, 576, 1, 16, None) == 1
+    assert lib.mla_absorb_q(g, g, g, g, 512, 1, 16, None) == 1      # ldq too small for q_rope
+    assert lib.mla_absorb_q(g, g, None, g, 516, 1, 16, None) == 1   # ldq not a multiple of 8
+    assert lib.mla_combine(None, g, 1, 16, 2, g, g, None) == 1
+    assert lib.mla_combine(g, g, 1, 16, 0, g, g, None) == 1

@@ -1,0 +1,185 @@
+"""GPU parity: mla_decode / mla_combine / mla_absorb_q through the C ABI
+against the FP64 oracle on the same seeded inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_latent_kv_25_b200 import binding, inputs
+from tests._util import assert_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def run(w, num_splits=0):
+    d = binding.to_device(w)
+    out, lse, ws = binding.decode_device(d, w.softmax_scale, num_splits=num_splits)
+    err = binding.mla_get_device_error(ws)
+    return out, lse, err
+
+
+def check_full(w, num_splits=0, what=""):
+    out, lse, err = run(w, num_splits)
+    assert err == 0, f"device error bits {err:#x}"
+    ro, rl = oracle.decode_workload(w)
+    assert_close(to_np(out).reshape(-1, 512), ro, what + " out")
+    assert_close(to_np(lse).reshape(-1), rl, what + " lse")
+    return out, lse
+
+
+# ---------------------------------------------------------------- small cases, every element
+
+def test_tiny_config_matches_oracle():
+    w = inputs.make("tiny")
+    check_full(w, what="tiny")
+
+
+@pytest.mark.parametrize("num_splits", [0, 1, 2, 3, 7, 64, 200])
+def test_ragged_small_all_split_counts(num_splits):
+    w = inputs.make("ragged", B=6, H=32, L=[1, 63, 64, 65, 1000, 130], seed=21, q_std=2.0,
+                    extra_blocks=4)
+    check_full(w, num_splits, what=f"splits={num_splits}")
+
+
+@pytest.mark.parametrize("H", [16, 48, 128])
+def test_head_counts(H):
+    w = inputs.make("v3", B=3, H=H, L=[300, 64, 129], seed=22, q_std=1.5)
+    check_full(w, what=f"H={H}")
+
+
+def test_sharp_softmax():
+    """Peaked rows (large query spread): errors in the scores show up here."""
+    w = inputs.make("v3", B=2, H=64, L=[777, 200], seed=23, q_std=6.0)
+    check_full(w, 5, what="sharp")
+
+
+def test_fp8_cache_small():
+    w = inputs.make("fp8", B=3, H=32, L=[200, 64, 1], seed=24, q_std=2.0, extra_blocks=2)
+    check_full(w, 3, what="fp8")
+
+
+@pytest.mark.parametrize("cache", ["bf16", "fp8"])
+def test_rows_past_seq_len_are_never_used(cache):
+    """NaN/huge values in the unused rows of each sequence's last block must
+    not reach the output."""
+    w = inputs.make("v3", B=3, H=16, L=[70, 130, 5], cache=cache, seed=25, tail_fill=float("nan"))
+    check_full(w, 2, what="tail-nan")
+    w = inputs.make("v3", B=3, H=16, L=[70, 130, 5], cache=cache, seed=25, tail_fill=3e38)
+    check_full(w, 0, what="tail-huge")
+
+
+def test_empty_sequences():
+    w = inputs.make("v3", B=4, H=16, L=[0, 100, 0, 64], seed=26)
+    out, lse = check_full(w, 3, what="empty")
+    o = to_np(out)
+    assert np.all(o[0] == 0) and np.all(o[2] == 0)
+    assert np.all(np.isneginf(to_np(lse)[[0, 2]]))
+
+
+@pytest.mark.parametrize("cache", ["bf16", "fp8"])
+@pytest.mark.parametrize("num_splits", [0, 5])
+def test_block_relocation_is_bit_exact(cache, num_splits):
+    """Physical placement of blocks must not change a single output bit."""
+    w = inputs.make("v3", B=3, H=32, L=[500, 64, 129], cache=cache, seed=27, extra_blocks=7)
+    w2 = inputs.relocate(w, seed=5)
+    o1, l1, e1 = run(w, num_splits)
+    o2, l2, e2 = run(w2, num_splits)
+    assert e1 == 0 and e2 == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1.view(torch.int32), l2.view(torch.int32))
+
+
+def test_constant_latent_column():
+    """Softmax weights sum to one: a latent column of ones reads back as 1."""
+    w = inputs.make("v3", B=2, H=32, L=[1000, 77], seed=28, q_std=3.0)
+    w.cache[:, :, 5] = 1.0
+    out, lse, err = run(w, 4)
+    assert err == 0
+    assert np.max(np.abs(to_np(out)[:, :, 5] - 1.0)) <= 2 ** -8
+
+
+def test_single_token_and_zero_query():
+    w = inputs.make("v3", B=2, H=16, L=[1, 64], seed=29)
+    w.q[1].zero_()
+    out, lse, err = run(w)
+    assert err == 0
+    row = w.cache[int(w.block_table[0, 0]), 0, :512].float().numpy()
+    assert np.max(np.abs(to_np(out)[0] - row[None])) <= 2 ** -8 * np.max(np.abs(row))
+    assert np.max(np.abs(to_np(lse)[1] - math.log(64))) < 1e-4
+
+
+# ---------------------------------------------------------------- device-side checks
+
+def test_bad_block_id_sets_error_bit():
+    w = inputs.make("v3", B=2, H=16, L=[100, 100], seed=30)
+    w.block_table[1, 1] = w.num_blocks + 5
+    out, lse, err = run(w)
+    assert err & binding.DEVERR_BAD_BLOCK
+
+
+def test_seq_len_beyond_table_sets_error_bit():
+    w = inputs.make("v3", B=2, H=16, L=[100, 100], seed=31)
+    w.seq_lens[0] = 64 * w.max_blocks + 1
+    out, lse, err = run(w)
+    assert err & binding.DEVERR_SEQ_TOO_LONG
+
+
+# ---------------------------------------------------------------- combine and absorb
+
+def test_combine_matches_oracle():
+    g = torch.Generator().manual_seed(32)
+    B, H, S = 3, 16, 5
+    o = torch.randn((B, H, S, 512), generator=g)
+    l = torch.randn((B, H, S), generator=g) * 3
+    l[0, 0, :] = -math.inf
+    l[1, 2, 1:] = -math.inf
+    out = torch.empty((B, H, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H), dtype=torch.float32, device="cuda")
+    binding.mla_combine(o.cuda(), l.cuda(), out, lse)
+    ro, rl = oracle.combine(o.double().reshape(B * H, S, 512).numpy(), l.double().reshape(B * H, S).numpy())
+    assert_close(to_np(out).reshape(-1, 512), ro, "combine out")
+    assert_close(to_np(lse).reshape(-1), rl, "combine lse", max_abs=1e-5)
+
+
+@pytest.mark.parametrize("B,H", [(1, 16), (5, 32), (64, 128)])
+def test_absorb_q_matches_oracle(B, H):
+    w = inputs.make("v3", B=B, H=H, L=[1] * B, seed=33)
+    qn, wu = w.q_nope.cuda(), w.w_uk.cuda()
+    qr = w.q[:, :, 512:].contiguous().cuda()
+    q_out = torch.zeros((B, H, 576), dtype=torch.bfloat16, device="cuda")
+    binding.mla_absorb_q(qn, wu, qr, q_out)
+    torch.cuda.synchronize()
+    ref = oracle.absorb_q(w.q_nope, w.w_uk)
+    assert_close(to_np(q_out[:, :, :512]).reshape(-1, 512), ref.reshape(-1, 512), "absorb")
+    assert torch.equal(q_out[:, :, 512:].cpu(), w.q[:, :, 512:])
+
+
+# ---------------------------------------------------------------- full-size configs, sampled rows
+
+def _sample_rows(w, n, seed):
+    rng = np.random.default_rng(seed)
+    nz = np.nonzero(w.seq_lens.numpy() > 0)[0]
+    b = rng.choice(nz, size=n, replace=True)
+    h = rng.integers(0, w.H, size=n)
+    rows = np.unique(np.stack([b, h], 1), axis=0)
+    # always include the longest sequence's first and last head
+    bl = int(np.argmax(w.seq_lens.numpy()))
+    return np.concatenate([rows, [[bl, 0], [bl, w.H - 1]]]).astype(np.int32)
+
+
+@pytest.mark.parametrize("name", ["v3", "ragged", "long", "fp8"])
+def test_full_config_sampled_rows(name):
+    w = inputs.make(name)
+    out, lse, err = run(w)
+    assert err == 0
+    rows = _sample_rows(w, 48 if name != "long" else 24, seed=1)
+    ro, rl = oracle.decode_workload(w, rows=rows)
+    o = to_np(out)[rows[:, 0], rows[:, 1]]
+    l = to_np(lse)[rows[:, 0], rows[:, 1]]
+    assert_close(o, ro, name + " out")
+    assert_close(l, rl, name + " lse")
+    # properties at full size: every row finite, lse >= max-free lower bound log(1)
+    assert np.all(np.isfinite(to_np(out)))
+    assert np.all(np.isfinite(to_np(lse)))
