@@ -39,7 +39,8 @@ __device__ __forceinline__ int clamp_len(int L, int max_blocks) {
 }
 
 // Iterates the segments of engine p.  Must be driven by a whole warp (all 32
-// lanes call the same methods); the returned values are warp-uniform.
+// lanes call the same methods); the returned values are warp-uniform.  With
+// NBt blocks in total only min(P, NBt) engines take part.
 struct SegWalker {
   const int32_t* seq_lens;
   int B, max_blocks, P, p;
@@ -57,13 +58,18 @@ struct SegWalker {
     P = P_;
     p = p_;
     NBt = warp_total_blocks(sl, B_, maxb);
-    s = range_start(p_, NBt, P_);
-    e = range_start(p_ + 1, NBt, P_);
+    // never more engines than blocks, so that every engine's range is
+    // non-empty and the engines holding one sequence are consecutive
+    if (static_cast<long long>(P) > NBt) P = static_cast<int>(NBt);
     count = 0;
     b = B;
     pre = 0;
     nb = 0;
     len = 0;
+    s = e = 0;
+    if (p >= P) return;
+    s = range_start(p_, NBt, P);
+    e = range_start(p_ + 1, NBt, P);
     if (s >= e) return;
     // find the sequence holding concatenated block s: warp scan over chunks of 32
     const int lane = threadIdx.x & 31;
