@@ -1,5 +1,6 @@
 // C ABI of libmla.so (declared in include/mla.h): host-side validation,
 // workspace layout, choice of the split-KV engine count, and the launches.
+#include <cudaTypedefs.h>
 #include <math.h>
 #include <mutex>
 
@@ -28,11 +29,57 @@ int device_sms() {
   return cache[dev];
 }
 
-// Engines of the split-KV partition: one per pair of SMs by default.
+// Clusters of the tensor-core decode that fit on the device at once.
+int device_max_clusters() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static std::mutex mu;
+  static int cache[64] = {0};
+  std::lock_guard<std::mutex> g(mu);
+  if (dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) cache[dev] = decode_sm100_max_clusters();
+  return cache[dev];
+}
+
+// Engines of the split-KV partition: by default one per co-resident cluster
+// of two SMs.
 int resolve_engines(int num_splits) {
   if (num_splits > 0) return num_splits;
   int sms = device_sms();
-  return sms >= 2 ? sms / 2 : 1;
+  if (sms < 2) return 0;
+  int P = sms / 2;
+  int mc = device_max_clusters();
+  if (mc > 0 && mc < P) P = mc;
+  return P;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 2-D view [rows, cols] of a row-major bf16 matrix, 64 x 64 box, 128 B swizzle.
+bool encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                     uint64_t row_bytes) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 constexpr int kMaxSplits = 4096;
@@ -132,7 +179,15 @@ mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void
   p.spin_limit = kDefaultSpin;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  cudaError_t e = launch_decode_simt(p, fp8, st);
+  cudaError_t e;
+  if (!fp8) {
+    CUtensorMap tmap;
+    if (!encode_bf16_map(&tmap, cache, uint64_t(num_blocks) * kBlock, kRow, kRow * 2))
+      return MLA_ERR_CUDA;
+    e = launch_decode_sm100(p, tmap, st);
+  } else {
+    e = launch_decode_simt(p, fp8, st);
+  }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   e = launch_merge_pieces(seq_lens, B, max_blocks_per_seq, H, p.seq_info, p.lse_part, p.o_part,
                           p.out, p.lse, p.err, st);

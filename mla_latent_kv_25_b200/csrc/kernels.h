@@ -1,6 +1,7 @@
 // Internal launch interface between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -26,8 +27,15 @@ struct DecodeParams {
   long long spin_limit;            // bounded-wait limit (clock64 cycles)
 };
 
-// CUDA-core scaffold decode (any H multiple of 16); fp8: cache is E4M3.
+// CUDA-core decode (any H multiple of 16); fp8: cache is E4M3.
 cudaError_t launch_decode_simt(const DecodeParams& p, bool fp8, cudaStream_t stream);
+
+// Tensor-core decode (bf16 cache): clusters of two CTAs, one engine each.
+// `tmap` is a 2-D tiled map over the cache viewed as [num_blocks*64, 576]
+// bf16 with a 64 x 64 box and 128-byte swizzle.
+cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, cudaStream_t stream);
+size_t decode_sm100_smem_bytes();
+int decode_sm100_max_clusters();
 
 cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H,
                                 const int4* seq_info, const float* lse_part, const float* o_part,
