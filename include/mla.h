@@ -146,6 +146,33 @@ mla_status_t mla_combine(const float *o_part, const float *lse_part, int B, int 
  */
 mla_status_t mla_get_device_error(void *workspace, void *stream, uint32_t *err_bits);
 
+/*
+ * mla_decode_noalloc - mla_decode with its scratch memory built into the
+ * library.  The paper has no counterpart: this is a deployment variant for
+ * callers that cannot allocate device memory themselves (processes that work
+ * inside a fixed budget carved out at start-up and route every later device
+ * allocation through their own pool, or latency-critical paths where
+ * cudaMalloc/cudaFree may synchronise the device).  Arguments are those of
+ * mla_decode without workspace/workspace_bytes; results are the same up to
+ * the last bits.
+ *
+ * Scratch: one file-scope device array of 40 MiB, held on every GPU that
+ * loads the library until the process exits.  A request whose scratch need
+ * (mla_decode_workspace_bytes(B, H, num_splits)) exceeds 40 MiB returns
+ * MLA_ERR_WORKSPACE_TOO_SMALL and launches nothing (at H = 128 the automatic
+ * split count of a B200 needs about 39 MB).  The first call on a device looks
+ * up the array's address on that device; make it before any stream capture.
+ * All calls on a device share the array and it keeps the last call's
+ * contents: calls that overlap on the GPU race, so serialise them.  Nothing
+ * in it needs clearing between calls.  Device-side error bits are recorded
+ * in the array but not reported.  Allocates and frees no device memory.
+ */
+mla_status_t mla_decode_noalloc(const void *q, mla_cache_dtype_t cache_dtype, const void *cache,
+                                const void *k_rope, const float *block_scale,
+                                const int32_t *block_table, const int32_t *seq_lens, int B, int H,
+                                int num_blocks, int max_blocks_per_seq, float softmax_scale,
+                                void *out, float *lse, int num_splits, void *stream);
+
 /* mla_status_string - a static, human-readable name for a status code. */
 const char *mla_status_string(mla_status_t status);
 

@@ -30,7 +30,7 @@ DEVERR_TIMEOUT = 0x4
 
 # every symbol include/mla.h declares
 EXPORTS = ("mla_absorb_q", "mla_decode_workspace_bytes", "mla_decode", "mla_combine",
-           "mla_get_device_error", "mla_status_string", "mla_num_sms")
+           "mla_get_device_error", "mla_status_string", "mla_num_sms", "mla_decode_noalloc")
 
 
 class MLAError(RuntimeError):
@@ -69,6 +69,9 @@ def load():
         L.mla_status_string.argtypes = [i32]
         L.mla_num_sms.restype = i32
         L.mla_num_sms.argtypes = []
+        L.mla_decode_noalloc.restype = i32
+        L.mla_decode_noalloc.argtypes = [vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                         ctypes.c_float, vp, vp, i32, vp]
         _lib = L
         return L
 
@@ -170,6 +173,27 @@ def mla_decode(q, cache, block_table, seq_lens, softmax_scale, out, lse, workspa
                            float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
                            int(workspace.numel()), int(num_splits), _stream(stream))
     _check("mla_decode", st)
+    return out, lse
+
+
+def mla_decode_noalloc(q, cache, block_table, seq_lens, softmax_scale, out, lse, *,
+                       k_rope=None, block_scale=None, num_splits=0, stream=None):
+    """mla_decode with the library's built-in scratch instead of a caller
+    workspace, for callers that cannot allocate device memory (see
+    include/mla.h): only inputs and outputs are passed."""
+    B, H = int(q.shape[0]), int(q.shape[1])
+    _need(q, "q", torch.bfloat16, (B, H, 576))
+    kind = MLA_CACHE_BF16 if cache.dtype == torch.bfloat16 else MLA_CACHE_FP8_E4M3
+    _need(cache, "cache", cache.dtype)
+    _need(block_table, "block_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    _need(out, "out", torch.bfloat16, (B, H, 512))
+    _need(lse, "lse", torch.float32, (B, H))
+    st = load().mla_decode_noalloc(_ptr(q), kind, _ptr(cache), _ptr(k_rope), _ptr(block_scale),
+                                   _ptr(block_table), _ptr(seq_lens), B, H, int(cache.shape[0]),
+                                   int(block_table.shape[1]), float(softmax_scale), _ptr(out),
+                                   _ptr(lse), int(num_splits), _stream(stream))
+    _check("mla_decode_noalloc", st)
     return out, lse
 
 
