@@ -4,21 +4,31 @@
 // role because the fp32 output accumulator of 128 heads x 512 latent columns
 // fills all 512 TMEM columns of one SM:
 //
-//   score CTA (rank 0)                         value CTA (rank 1)
-//   -----------------                          -----------------
-//   w0  TMA: cache rows [64 x 576] -> smem      w0  TMA: latent part [64 x 512] -> smem
-//   w1  MMA: S = Q K^T  (A = Q in TMEM,          w1  MMA: O += P V  (A = P, B = V, both
-//       B = K tile, N = 64 tokens, K = 576)          smem; V read MN-major from the tile)
-//   w4-7 softmax, thread h = head h: online     w2  zero rows past seq_len in the V tile
-//       softmax in fp32, P (bf16) and the        w4-7 thread h = head h: rescale O rows when
-//       rescale factors to the value CTA             the running max grew, final O / l and
-//       by a bulk shared->shared copy                lse (or an fp32 piece of a cut sequence)
+//   score CTA (rank 0)                           value CTA (rank 1)
+//   ------------------                           ------------------
+//   w0  TMA: cache rows of two 64-token blocks    w0  TMA: latent part of each block,
+//       per pass, one 64-column chunk at a time       half a block (4 chunks) at a time
+//       into a ring of [128 x 64] slots               into a ring of [64 x 256] slots
+//   w1  MMA: S = Q K^T for 128 tokens at once     w1  MMA: O += P V (A = P, B = V read
+//       (N = 128); latent part of Q in TMEM,          MN-major), N = 256 per instruction
+//       RoPE part of Q in shared memory           w2  zero V rows past seq_len
+//   w4-7 softmax, thread h = head h: online       w4-7 thread h = head h: rescale O rows
+//       softmax in fp32 per 64-token block;           when the running max grew; final
+//       P (bf16) and the rescale factors are         O / l and lse, or an fp32 piece of
+//       staged locally                                a cut sequence
+//   w2-3 senders: staged records -> value CTA
+//       with st.async (overlapping the softmax)
 //
-// Heads are the M = 128 dimension of both contractions (padded with zero
-// query rows for H < 128).  The running max is only moved when a block's max
-// exceeds it by more than 2^8 (log2 domain), so O is rarely rescaled.
-// Every wait is bounded (WaitCtx); a timeout records an error bit and the
-// CTA leaves its loops, releases TMEM and exits.
+// Heads are the M = 128 dimension of both contractions (padded with zero query
+// rows for H < 128).  The running max only moves when a block's max exceeds
+// it by more than 2^8 (log2 domain), so O is rarely rescaled.  Every wait is
+// bounded (WaitCtx); a timeout records an error bit and the CTA leaves its
+// loops, releases TMEM and exits.
+//
+// Barrier discipline: a parity wait can only tell the current phase from the
+// one before it, so every barrier here is either observed by its waiters at
+// every phase, in order, or used as a strict two-party handshake (q_ready /
+// q_free, pv_prev / corr_done, o_ready / o_free).
 #include <cuda.h>
 #include <math.h>
 
@@ -33,33 +43,36 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 256;
-constexpr int kNK = 2;  // K-tile stages (score CTA)
-constexpr int kNV = 2;  // V-tile stages (value CTA)
-constexpr int kNP = 2;  // P records in flight
-constexpr int kNS = 3;  // S accumulators in TMEM
+constexpr int kKSlots = 9;   // score CTA: ring of [128 tokens x 64 cols] chunk slots
+constexpr int kVSlots = 5;   // value CTA: ring of [64 tokens x 256 cols] half-block slots
+constexpr int kNP = 3;       // P records in flight
+constexpr int kNS = 2;       // S accumulators (128 columns each) in TMEM
 
-constexpr uint32_t kChunk = 64 * 128;                  // one [64 rows x 64 bf16] swizzled chunk
-constexpr uint32_t kKStage = 9 * kChunk;               // 73728 B: rows [c_kv | k_rope]
-constexpr uint32_t kVStage = 8 * kChunk;               // 65536 B: c_kv part only
-constexpr uint32_t kPBytes = 128 * 64 * 2;             // P [128 heads x 64 tokens] bf16
-constexpr uint32_t kPWarpBytes = 32 * 128;             // one warp's 32 rows of P
-constexpr uint32_t kMetaWarp = 400;                    // per warp: alpha[32] m[32] l[32] flag + pad
+constexpr uint32_t kChunk = 64 * 128;          // one [64 rows x 64 bf16] swizzled chunk
+constexpr uint32_t kKSlot = 2 * kChunk;         // [128 rows x 64 bf16]
+constexpr uint32_t kVSlot = 4 * kChunk;         // [64 rows x 256 bf16]
+constexpr uint32_t kPBytes = 128 * 64 * 2;     // P [128 heads x 64 tokens] bf16
+constexpr uint32_t kQRopeBytes = 128 * 64 * 2; // RoPE part of Q [128 heads x 64] bf16
+constexpr uint32_t kMetaWarp = 400;            // per warp: alpha[32] m[32] l[32] flag + pad
 constexpr uint32_t kMetaBytes = 4 * kMetaWarp;
-constexpr float kRescaleThreshold = 8.0f;              // log2 units
+constexpr float kRescaleThreshold = 8.0f;      // log2 units
+constexpr int kPrefetchAhead = 8;              // blocks prefetched into L2 ahead of the K ring
+constexpr float kLog2e = 1.4426950408889634f;
 
-// TMEM columns
-constexpr uint32_t kQCol = 0;      // score CTA: Q, 576 bf16 = 288 columns
-constexpr uint32_t kSCol = 288;    // score CTA: S buffers, 64 columns each
+// TMEM columns of the score CTA: latent part of Q (512 bf16 = 256 columns), then S.
+constexpr uint32_t kQCol = 0;
+constexpr uint32_t kSCol = 256;
 constexpr uint32_t kTmemCols = 512;
 
 struct Barriers {
-  uint64_t k_full[kNK], k_empty[kNK];
+  uint64_t k_full[kKSlots], k_empty[kKSlots];
   uint64_t s_full[kNS], s_empty[kNS];
   uint64_t q_ready, q_free;
   uint64_t p_empty[kNP];
-  uint64_t v_full[kNV], v_empty[kNV], v_fixed[kNV];
+  uint64_t stage_full[kNP], stage_empty[kNP];
+  uint64_t v_full[kVSlots], v_empty[kVSlots], v_fixed[kVSlots];
   uint64_t p_full[kNP];
-  uint64_t pv_done, corr_done, o_free;
+  uint64_t pv_prev, corr_done, o_ready, o_free;
   uint32_t tmem_base;
   int abort;
 };
@@ -67,29 +80,32 @@ static_assert(sizeof(Barriers) <= 1024, "barrier block too large");
 
 // shared-memory offsets from the 1024-aligned base
 constexpr uint32_t kRegion = 1024;
-__host__ __device__ constexpr uint32_t k_stage_off(int s) { return kRegion + s * kKStage; }
-__host__ __device__ constexpr uint32_t p_stage_off(int r) { return kRegion + kNK * kKStage + r * kPBytes; }
+__host__ __device__ constexpr uint32_t q_rope_off() { return kRegion; }
+__host__ __device__ constexpr uint32_t k_slot_off(int s) { return kRegion + kQRopeBytes + s * kKSlot; }
+// score CTA staging of the P records and factors before the bulk copy
+__host__ __device__ constexpr uint32_t p_stage_off(int r) { return k_slot_off(kKSlots) + r * kPBytes; }
 __host__ __device__ constexpr uint32_t meta_stage_off(int r) {
-  return kRegion + kNK * kKStage + kNP * kPBytes + r * kMetaBytes;
+  return k_slot_off(kKSlots) + kNP * kPBytes + r * kMetaBytes;
 }
-__host__ __device__ constexpr uint32_t v_stage_off(int s) { return kRegion + s * kVStage; }
-__host__ __device__ constexpr uint32_t p_rec_off(int r) { return kRegion + kNV * kVStage + r * kPBytes; }
+__host__ __device__ constexpr uint32_t v_slot_off(int s) { return kRegion + s * kVSlot; }
+__host__ __device__ constexpr uint32_t p_rec_off(int r) { return kRegion + kVSlots * kVSlot + r * kPBytes; }
 __host__ __device__ constexpr uint32_t meta_rec_off(int r) {
-  return kRegion + kNV * kVStage + kNP * kPBytes + r * kMetaBytes;
+  return kRegion + kVSlots * kVSlot + kNP * kPBytes + r * kMetaBytes;
 }
 constexpr uint32_t kScoreSmem = meta_stage_off(kNP);
 constexpr uint32_t kValueSmem = meta_rec_off(kNP);
 constexpr uint32_t kSmemBytes = (kScoreSmem > kValueSmem ? kScoreSmem : kValueSmem) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(p_stage_off(0) % 1024 == 0 && p_rec_off(0) % 1024 == 0, "swizzle atoms need 1024 B");
+static_assert(k_slot_off(0) % 1024 == 0 && p_rec_off(0) % 1024 == 0 && p_stage_off(0) % 1024 == 0,
+              "swizzle atoms need 1024 B");
 
-constexpr uint32_t kIdescQK = idesc_bf16(128, 64, false, false);   // S[128x64] = Q . K^T
+constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false, false);  // S[128x128] = Q . K^T
 constexpr uint32_t kIdescPV = idesc_bf16(128, 256, false, true);   // O[128x256] += P . V
 
 struct Ctx {
   const DecodeParams* p;
-  uint32_t base;        // shared address of the aligned base
-  uint8_t* gbase;       // generic pointer to it
+  uint32_t base;   // shared address of the aligned base
+  uint8_t* gbase;  // generic pointer to it
   Barriers* bars;
   uint32_t tmem;
   WaitCtx wc;
@@ -97,20 +113,38 @@ struct Ctx {
   int warp, lane;
 };
 
-__device__ __forceinline__ uint32_t bar_addr(const Ctx& c, const uint64_t& b) { return smem_u32(&b); }
+__device__ __forceinline__ uint32_t bar_addr(const uint64_t& b) { return smem_u32(&b); }
 
-// all lanes wait; the warp proceeds only if every lane saw the phase complete
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
-  bool ok = wait_phase(bar, parity, w);
-  return __all_sync(0xffffffffu, ok);
-}
+// Physical block ids of one sequence, fetched 32 at a time by the whole warp
+// (one global load per 32 blocks instead of one per block).
+struct BlockCursor {
+  const int32_t* row;
+  int nblk;
+  int base;
+  int cached;
+
+  __device__ void reset(const DecodeParams& p, const Segment& g) {
+    row = p.block_table + size_t(g.b) * p.max_blocks;
+    nblk = nblocks_of(g.len);
+    base = -64;
+    cached = -1;
+  }
+  // id of logical block j (warp-uniform j < nblk)
+  __device__ int id(int j, int lane) {
+    if (j < base || j >= base + 32) {
+      base = j;
+      cached = (j + lane < nblk) ? row[j + lane] : -1;
+    }
+    return __shfl_sync(0xffffffffu, cached, j - base);
+  }
+};
 
 // Valid rows of logical block j of segment g (0 for an out-of-range block id);
 // *blk receives a block that is safe to load.
-__device__ __forceinline__ int block_rows(const DecodeParams& p, const Segment& g, int j,
-                                          int* blk) {
-  int id = p.block_table[size_t(g.b) * p.max_blocks + j];
-  bool ok = id >= 0 && id < p.num_blocks;
+__device__ __forceinline__ int block_rows(const DecodeParams& p, const Segment& g, BlockCursor& cur,
+                                          int j, int lane, int* blk) {
+  const int id = cur.id(j, lane);
+  const bool ok = id >= 0 && id < p.num_blocks;
   *blk = ok ? id : 0;
   int nv = g.len - j * kBlock;
   nv = nv > kBlock ? kBlock : nv;
@@ -119,40 +153,71 @@ __device__ __forceinline__ int block_rows(const DecodeParams& p, const Segment& 
 
 // ============================================================ score CTA roles
 
+// Two consecutive blocks of a segment form one pass (the second may be
+// absent at the end of the segment); each pass streams its 9 column chunks
+// through the slot ring.
 __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   const DecodeParams& p = *c.p;
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
-  uint32_t it = 0;
+  BlockCursor cur;
+  uint32_t cit = 0;
   bool alive = true;
   if (c.lane == 0) prefetch_tmap(tmap);
+  const uint8_t* cache = static_cast<const uint8_t*>(p.cache);
+  BlockCursor pcur;  // block ids for the L2 prefetch, kPrefetchAhead blocks ahead
   while (alive && w.next(g)) {
-    for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
-      const int s = it % kNK;
-      const uint32_t ph = (it / kNK) & 1u;
-      if (!warp_wait(bar_addr(c, c.bars->k_empty[s]), ph ^ 1u, c.wc)) {
-        alive = false;
-        break;
+    cur.reset(p, g);
+    pcur.reset(p, g);
+    // warm L2 with the first blocks of the segment; from then on each pass
+    // prefetches the two blocks kPrefetchAhead ahead, so the ring's TMA loads
+    // hit L2 (the ring itself is too small to cover HBM latency)
+    for (int j = g.blk_lo; j < g.blk_lo + kPrefetchAhead && j < g.blk_hi; ++j) {
+      int pb;
+      const int nv = block_rows(p, g, pcur, j, c.lane, &pb);
+      if (c.lane == 0 && nv > 0) prefetch_l2_bulk(cache + size_t(pb) * kBlock * kRow * 2, kBlock * kRow * 2);
+    }
+    for (int j = g.blk_lo; alive && j < g.blk_hi; j += 2) {
+      for (int q = 0; q < 2; ++q) {
+        const int jp = j + kPrefetchAhead + q;
+        if (jp < g.blk_hi) {
+          int pb;
+          const int nv = block_rows(p, g, pcur, jp, c.lane, &pb);
+          if (c.lane == 0 && nv > 0) prefetch_l2_bulk(cache + size_t(pb) * kBlock * kRow * 2, kBlock * kRow * 2);
+        }
       }
-      int blk;
-      const int nv = block_rows(p, g, j, &blk);
+      int blk_a, blk_b = 0;
+      const int nv_a = block_rows(p, g, cur, j, c.lane, &blk_a);
+      const bool has_b = j + 1 < g.blk_hi;
+      int nv_b = 0;
+      if (has_b) nv_b = block_rows(p, g, cur, j + 1, c.lane, &blk_b);
       if (c.lane == 0) {
-        if (nv == 0 && g.len > j * kBlock) atomicOr(p.err, kErrBadBlock);
-        const uint32_t full = bar_addr(c, c.bars->k_full[s]);
-        mbar_arrive_expect_tx(full, kKStage);
-        const uint32_t dst = c.base + k_stage_off(s);
-#pragma unroll
-        for (int ch = 0; ch < 9; ++ch) tma_load_2d(dst + ch * kChunk, tmap, ch * 64, blk * kBlock, full);
+        if (nv_a == 0 && g.len > j * kBlock) atomicOr(p.err, kErrBadBlock);
+        if (has_b && nv_b == 0) atomicOr(p.err, kErrBadBlock);
       }
-      __syncwarp();
+      for (int ch = 0; ch < 9; ++ch, ++cit) {
+        const int s = cit % kKSlots;
+        if (!warp_wait(bar_addr(c.bars->k_empty[s]), ((cit / kKSlots) & 1u) ^ 1u, c.wc)) {
+          alive = false;
+          break;
+        }
+        if (c.lane == 0) {
+          const uint32_t full = bar_addr(c.bars->k_full[s]);
+          mbar_arrive_expect_tx(full, has_b ? kKSlot : kChunk);
+          const uint32_t dst = c.base + k_slot_off(s);
+          tma_load_2d(dst, tmap, ch * 64, blk_a * kBlock, full);
+          if (has_b) tma_load_2d(dst + kChunk, tmap, ch * 64, blk_b * kBlock, full);
+        }
+        __syncwarp();
+      }
     }
   }
-  // wait for the loads this warp issued (bounded) before the CTA may exit
+  // wait (bounded) for the loads this warp issued before the CTA may exit
   if (!alive) {
-    for (uint32_t k = (it > kNK ? it - kNK : 0); k < it; ++k) {
+    for (uint32_t k = (cit > kKSlots ? cit - kKSlots : 0); k < cit; ++k) {
       const long long t0 = clock64();
-      while (!mbar_try_wait(bar_addr(c, c.bars->k_full[k % kNK]), (k / kNK) & 1u) &&
+      while (!mbar_try_wait(bar_addr(c.bars->k_full[k % kKSlots]), (k / kKSlots) & 1u) &&
              clock64() - t0 < 2000000000LL) {
       }
     }
@@ -164,33 +229,160 @@ __device__ void score_mma(const Ctx& c) {
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
-  uint32_t it = 0, seg = 0;
+  uint32_t cit = 0, pit = 0, seg = 0;
+  const uint32_t qrope = c.base + q_rope_off();
   while (w.next(g)) {
-    if (!warp_wait(bar_addr(c, c.bars->q_ready), seg & 1u, c.wc)) return;
+    if (!warp_wait(bar_addr(c.bars->q_ready), seg & 1u, c.wc)) return;
     tc_fence_after();
-    for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
-      const int s = it % kNK;
-      const int sb = it % kNS;
-      if (!warp_wait(bar_addr(c, c.bars->k_full[s]), (it / kNK) & 1u, c.wc)) return;
-      if (!warp_wait(bar_addr(c, c.bars->s_empty[sb]), ((it / kNS) & 1u) ^ 1u, c.wc)) return;
-      tc_fence_after();
-      if (c.lane == 0) {
-        const uint32_t d = c.tmem + kSCol + sb * 64;
-        const uint32_t kst = c.base + k_stage_off(s);
-#pragma unroll 4
-        for (int k = 0; k < kRow / 16; ++k) {
-          const uint32_t b_addr = kst + (k >> 2) * kChunk + (k & 3) * 32;
-          mma_ts(d, c.tmem + kQCol + 8 * k, sw128_desc(b_addr, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+    for (int j = g.blk_lo; j < g.blk_hi; j += 2, ++pit) {
+      const int sb = pit % kNS;
+      if (!warp_wait(bar_addr(c.bars->s_empty[sb]), ((pit / kNS) & 1u) ^ 1u, c.wc)) return;
+      const uint32_t d = c.tmem + kSCol + sb * 128;
+      for (int ch = 0; ch < 9; ++ch, ++cit) {
+        const int s = cit % kKSlots;
+        if (!warp_wait(bar_addr(c.bars->k_full[s]), (cit / kKSlots) & 1u, c.wc)) return;
+        tc_fence_after();
+        if (c.lane == 0) {
+          const uint32_t slot = c.base + k_slot_off(s);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t b = sw128_desc(slot + kk * 32, 16, 1024);
+            if (ch < 8)
+              mma_ts(d, c.tmem + kQCol + 32 * ch + 8 * kk, b, kIdescQK, (ch | kk) ? 1u : 0u);
+            else
+              mma_ss(d, sw128_desc(qrope + kk * 32, 16, 1024), b, kIdescQK, 1u);
+          }
+          mma_commit(bar_addr(c.bars->k_empty[s]));
         }
-        mma_commit(bar_addr(c, c.bars->k_empty[s]));
-        mma_commit(bar_addr(c, c.bars->s_full[sb]));
+        __syncwarp();
       }
+      if (c.lane == 0) mma_commit(bar_addr(c.bars->s_full[sb]));
       __syncwarp();
     }
-    if (c.lane == 0) mma_commit(bar_addr(c, c.bars->q_free));
+    if (c.lane == 0) mma_commit(bar_addr(c.bars->q_free));
     __syncwarp();
     ++seg;
   }
+}
+
+// Query row of sequence b for head h: the latent part (512 bf16) into TMEM
+// lane h as 256 packed columns, the RoPE part (64 bf16) into the swizzled
+// [128 x 64] K-major tile in shared memory.  Loads run four chunks ahead.
+__device__ __forceinline__ void load_q_rows(const DecodeParams& p, int b, int h, uint32_t taddr,
+                                            uint8_t* qrope) {
+  const bool live = h < p.H;
+  const uint4* src = reinterpret_cast<const uint4*>(p.q + (size_t(b) * p.H + (live ? h : 0)) * kRow);
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  uint4 rope[8];
+#pragma unroll
+  for (int v = 0; v < 8; ++v) rope[v] = live ? __ldg(src + 64 + v) : z;
+  uint4 buf[4][8];
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+    for (int v = 0; v < 8; ++v) buf[ch][v] = live ? __ldg(src + ch * 8 + v) : z;
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch) {
+    uint32_t r[32];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      r[4 * v] = buf[ch % 4][v].x;
+      r[4 * v + 1] = buf[ch % 4][v].y;
+      r[4 * v + 2] = buf[ch % 4][v].z;
+      r[4 * v + 3] = buf[ch % 4][v].w;
+    }
+    tmem_st32(taddr + 32 * ch, r);
+    if (ch + 4 < 8) {
+#pragma unroll
+      for (int v = 0; v < 8; ++v) buf[ch % 4][v] = live ? __ldg(src + (ch + 4) * 8 + v) : z;
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    *reinterpret_cast<uint4*>(qrope + h * 128 + ((v ^ (h & 7)) << 4)) = rope[v];
+}
+
+__device__ __forceinline__ void prefetch_q_rows_l2(const DecodeParams& p, int b, int h) {
+  if (h >= p.H) return;
+  const char* src = reinterpret_cast<const char*>(p.q + (size_t(b) * p.H + h) * kRow);
+#pragma unroll
+  for (int i = 0; i < 9; ++i) asm volatile("prefetch.global.L2 [%0];" ::"l"(src + 128 * i));
+}
+
+struct SoftmaxState {
+  float m_ref, l;
+};
+
+// Online softmax of one 64-token block (raw scores in sv) and its hand-off to
+// the value CTA.  Returns false if a wait gave up.
+__device__ __forceinline__ bool softmax_block(const Ctx& c, const uint32_t (&sv)[64], int nv, bool first,
+                                              float sl2, bool pos, SoftmaxState& st, uint32_t it,
+                                              int h, int q4) {
+  // block max of the scaled scores (the sign of the scale decides max or min)
+  float mr;
+  if (nv == kBlock) {
+    mr = __uint_as_float(sv[0]);
+#pragma unroll
+    for (int t = 1; t < 64; ++t) mr = pos ? fmaxf(mr, __uint_as_float(sv[t])) : fminf(mr, __uint_as_float(sv[t]));
+  } else {
+    mr = pos ? -INFINITY : INFINITY;
+#pragma unroll
+    for (int t = 0; t < 64; ++t)
+      if (t < nv) mr = pos ? fmaxf(mr, __uint_as_float(sv[t])) : fminf(mr, __uint_as_float(sv[t]));
+  }
+  const float mx = nv > 0 ? mr * sl2 : -INFINITY;
+  float alpha = 1.f;
+  bool resc = false;
+  if (first) {
+    st.m_ref = mx;
+  } else if (mx > st.m_ref + kRescaleThreshold) {
+    alpha = (st.m_ref == -INFINITY) ? 0.f : ex2_approx(st.m_ref - mx);
+    st.m_ref = mx;
+    st.l *= alpha;
+    resc = true;
+  }
+  const float neg_m = st.m_ref == -INFINITY ? 0.f : -st.m_ref;
+  uint32_t pk[32];
+  float sum = 0.f;
+  if (nv == kBlock) {
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const float e0 = ex2_approx(fmaf(__uint_as_float(sv[2 * t]), sl2, neg_m));
+      const float e1 = ex2_approx(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, neg_m));
+      sum += e0 + e1;
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+      pk[t] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const float e0 = 2 * t < nv ? ex2_approx(fmaf(__uint_as_float(sv[2 * t]), sl2, neg_m)) : 0.f;
+      const float e1 = 2 * t + 1 < nv ? ex2_approx(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, neg_m)) : 0.f;
+      sum += e0 + e1;
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+      pk[t] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+  }
+  st.l += sum;
+
+  // P row and the per-head factors into this CTA's staging record r; the
+  // sender warps move it to the value CTA
+  const int r = it % kNP;
+  if (!warp_wait(bar_addr(c.bars->stage_empty[r]), ((it / kNP) & 1u) ^ 1u, c.wc)) return false;
+  uint8_t* prow = c.gbase + p_stage_off(r) + h * 128;
+  const uint32_t swz = static_cast<uint32_t>(h & 7);
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch)
+    *reinterpret_cast<uint4*>(prow + ((static_cast<uint32_t>(ch) ^ swz) << 4)) =
+        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+  float* meta = reinterpret_cast<float*>(c.gbase + meta_stage_off(r) + q4 * kMetaWarp);
+  meta[c.lane] = alpha;
+  meta[32 + c.lane] = st.m_ref;
+  meta[64 + c.lane] = st.l;
+  const unsigned any = __any_sync(0xffffffffu, resc);
+  if (c.lane == 0) reinterpret_cast<uint32_t*>(meta)[96] = any ? 1u : 0u;
+  mbar_arrive(bar_addr(c.bars->stage_full[r]));
+  return true;
 }
 
 __device__ void score_softmax(const Ctx& c) {
@@ -198,127 +390,121 @@ __device__ void score_softmax(const Ctx& c) {
   const int q4 = c.warp - 4;              // TMEM lane quadrant
   const int h = q4 * 32 + c.lane;         // head of this thread
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-  const float sl2 = p.softmax_scale * 1.4426950408889634f;
+  const float sl2 = p.softmax_scale * kLog2e;
+  const bool pos = sl2 >= 0.f;
+  uint8_t* qrope = c.gbase + q_rope_off();
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
-  uint32_t it = 0, seg = 0, pit = 0;
+  BlockCursor cur;
+  uint32_t it = 0, pit = 0, seg = 0;
   bool alive = true;
   while (alive && w.next(g)) {
-    // ---- this sequence's query row into TMEM (A operand of Q K^T)
+    cur.reset(p, g);
     if (seg > 0) {
-      if (!warp_wait(bar_addr(c, c.bars->q_free), (seg - 1) & 1u, c.wc)) break;
+      if (!warp_wait(bar_addr(c.bars->q_free), (seg - 1) & 1u, c.wc)) break;
       tc_fence_after();
     }
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(p.q + (size_t(g.b) * p.H + h) * kRow);
-      const bool live = h < p.H;
-#pragma unroll 1
-      for (int ch = 0; ch < 9; ++ch) {
-        uint32_t r[32];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          uint4 x = live ? __ldg(src + ch * 8 + v) : make_uint4(0, 0, 0, 0);
-          r[4 * v] = x.x;
-          r[4 * v + 1] = x.y;
-          r[4 * v + 2] = x.z;
-          r[4 * v + 3] = x.w;
-        }
-        tmem_st32(c.tmem + lane_off + kQCol + 32 * ch, r);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar_addr(c, c.bars->q_ready));
-    }
-    float m_ref = -INFINITY, l = 0.f;
-    for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it, ++pit) {
+    load_q_rows(p, g.b, h, c.tmem + lane_off + kQCol, qrope);
+    fence_proxy_async_smem();
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(bar_addr(c.bars->q_ready));
+    if (w.b < w.B && w.pre < w.e) prefetch_q_rows_l2(p, w.b, h);  // next segment's query
+
+    SoftmaxState st{-INFINITY, 0.f};
+    for (int j = g.blk_lo; j < g.blk_hi; j += 2, ++pit) {
+      const int sb = pit % kNS;
+      const bool has_b = j + 1 < g.blk_hi;
       int blk;
-      const int nv = block_rows(p, g, j, &blk);
-      const int sb = it % kNS;
-      if (!warp_wait(bar_addr(c, c.bars->s_full[sb]), (it / kNS) & 1u, c.wc)) {
+      const int nv_a = block_rows(p, g, cur, j, c.lane, &blk);
+      const int nv_b = has_b ? block_rows(p, g, cur, j + 1, c.lane, &blk) : 0;
+      if (!warp_wait(bar_addr(c.bars->s_full[sb]), (pit / kNS) & 1u, c.wc)) {
         alive = false;
         break;
       }
       tc_fence_after();
-      uint32_t s0[32], s1[32];
-      tmem_ld32(c.tmem + lane_off + kSCol + sb * 64, s0);
-      tmem_ld32(c.tmem + lane_off + kSCol + sb * 64 + 32, s1);
+      const uint32_t sa = c.tmem + lane_off + kSCol + sb * 128;
+      uint32_t sv[64];
+      tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar_addr(c, c.bars->s_empty[sb]));
-
-      float x[64];
-#pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        x[t] = t < nv ? __uint_as_float(s0[t]) * sl2 : -INFINITY;
-        x[t + 32] = t + 32 < nv ? __uint_as_float(s1[t]) * sl2 : -INFINITY;
+      if (!has_b) {
+        tc_fence_before();
+        mbar_arrive(bar_addr(c.bars->s_empty[sb]));
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int t = 0; t < 64; ++t) mx = fmaxf(mx, x[t]);
-      const bool first = (j == g.blk_lo);
-      const bool last = (j == g.blk_hi - 1);
-      float alpha = 1.f;
-      bool resc = false;
-      if (first) {
-        m_ref = mx;
-      } else if (mx > m_ref + kRescaleThreshold) {
-        alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
-        m_ref = mx;
-        l *= alpha;
-        resc = true;
-      }
-      uint32_t pk[32];
-      float sum = 0.f;
-#pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const float e0 = x[2 * t] == -INFINITY ? 0.f : exp2f(x[2 * t] - m_ref);
-        const float e1 = x[2 * t + 1] == -INFINITY ? 0.f : exp2f(x[2 * t + 1] - m_ref);
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
-        const float2 rb = __bfloat1622float2(b2);
-        sum += rb.x + rb.y;
-        pk[t] = *reinterpret_cast<uint32_t*>(&b2);
-      }
-      l += sum;
-
-      // ---- ship P and the per-head factors to the value CTA
-      const int r = pit % kNP;
-      if (!warp_wait(bar_addr(c, c.bars->p_empty[r]), ((pit / kNP) & 1u) ^ 1u, c.wc)) {
+      if (!softmax_block(c, sv, nv_a, j == g.blk_lo, sl2, pos, st, it, h, q4)) {
         alive = false;
         break;
       }
-      uint8_t* prow = c.gbase + p_stage_off(r) + h * 128;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (h & 7)) << 4)) = v;
+      ++it;
+      if (has_b) {
+        tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(bar_addr(c.bars->s_empty[sb]));
+        if (!softmax_block(c, sv, nv_b, false, sl2, pos, st, it, h, q4)) {
+          alive = false;
+          break;
+        }
+        ++it;
       }
-      float* meta = reinterpret_cast<float*>(c.gbase + meta_stage_off(r) + q4 * kMetaWarp);
-      meta[c.lane] = alpha;
-      meta[32 + c.lane] = m_ref;
-      meta[64 + c.lane] = l;
-      const unsigned any = __any_sync(0xffffffffu, resc);
-      if (c.lane == 0) reinterpret_cast<uint32_t*>(meta)[96] = any ? 1u : 0u;
-      (void)last;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (c.lane == 0) {
-        const uint32_t full = bar_addr(c, c.bars->p_full[r]);
-        mbar_arrive_expect_tx_remote(full, 1, kPWarpBytes + kMetaWarp);
-        bulk_copy_to_rank(c.base + p_rec_off(r) + q4 * kPWarpBytes,
-                          c.base + p_stage_off(r) + q4 * kPWarpBytes, kPWarpBytes, full, 1);
-        bulk_copy_to_rank(c.base + meta_rec_off(r) + q4 * kMetaWarp,
-                          c.base + meta_stage_off(r) + q4 * kMetaWarp, kMetaWarp, full, 1);
-      }
-      __syncwarp();
     }
     ++seg;
+  }
+  (void)alive;
+}
+
+// Sender warps (2 and 3 of the score CTA): copy each staged record into the
+// value CTA with st.async (register -> remote shared memory, bytes counted on
+// its p_full[r]) so that the slow SM-to-SM transfer overlaps the softmax of
+// the next block.
+constexpr uint32_t kRecUnits = (kPBytes + kMetaBytes) / 16;  // 16-byte units per record
+
+__device__ void score_sender(const Ctx& c) {
+  const DecodeParams& p = *c.p;
+  const int sid = (c.warp - 2) * 32 + c.lane;  // 0..63
+  const uint32_t prec0 = map_to_rank(c.base + p_rec_off(0), 1);
+  const uint32_t mrec0 = map_to_rank(c.base + meta_rec_off(0), 1);
+  const uint32_t pfull0 = map_to_rank(bar_addr(c.bars->p_full[0]), 1);
+  uint32_t my_units = 0;
+  for (uint32_t u = sid; u < kRecUnits; u += 64) ++my_units;
+  SegWalker w;
+  w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
+  Segment g;
+  uint32_t it = 0;
+  bool alive = true;
+  while (alive && w.next(g)) {
+    for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
+      const int r = it % kNP;
+      if (!warp_wait(bar_addr(c.bars->stage_full[r]), (it / kNP) & 1u, c.wc) ||
+          !warp_wait(bar_addr(c.bars->p_empty[r]), ((it / kNP) & 1u) ^ 1u, c.wc)) {
+        alive = false;
+        break;
+      }
+      const uint32_t fullr = pfull0 + 8 * r;
+      mbar_arrive_expect_tx_cluster_relaxed(fullr, my_units * 16);
+      const uint8_t* pst = c.gbase + p_stage_off(r);
+      const uint8_t* mst = c.gbase + meta_stage_off(r);
+      for (uint32_t u = sid; u < kRecUnits; u += 64) {
+        if (u < kPBytes / 16) {
+          const uint4 v = *reinterpret_cast<const uint4*>(pst + u * 16);
+          st_async_v4(prec0 + r * kPBytes + u * 16, v, fullr);
+        } else {
+          const uint32_t m = u - kPBytes / 16;
+          const uint4 v = *reinterpret_cast<const uint4*>(mst + m * 16);
+          st_async_v4(mrec0 + r * kMetaBytes + m * 16, v, fullr);
+        }
+      }
+      mbar_arrive(bar_addr(c.bars->stage_empty[r]));
+    }
   }
   // drain: every record handed to the value CTA has been released, so no
   // remote arrival on this CTA is still pending when it exits
   if (alive) {
-    for (uint32_t k = (pit > kNP ? pit - kNP : 0); k < pit; ++k)
-      if (!warp_wait(bar_addr(c, c.bars->p_empty[k % kNP]), (k / kNP) & 1u, c.wc)) break;
+    for (uint32_t k = (it > kNP ? it - kNP : 0); k < it; ++k)
+      if (!warp_wait(bar_addr(c.bars->p_empty[k % kNP]), (k / kNP) & 1u, c.wc)) break;
   }
 }
 
@@ -329,68 +515,76 @@ __device__ void value_tma(const Ctx& c, const CUtensorMap* tmap) {
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
-  uint32_t it = 0;
+  BlockCursor cur;
+  uint32_t vit = 0;
   bool alive = true;
   if (c.lane == 0) prefetch_tmap(tmap);
   while (alive && w.next(g)) {
-    for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
-      const int s = it % kNV;
-      if (!warp_wait(bar_addr(c, c.bars->v_empty[s]), ((it / kNV) & 1u) ^ 1u, c.wc)) {
-        alive = false;
-        break;
-      }
+    cur.reset(p, g);
+    for (int j = g.blk_lo; alive && j < g.blk_hi; ++j) {
       int blk;
-      block_rows(p, g, j, &blk);
-      if (c.lane == 0) {
-        const uint32_t full = bar_addr(c, c.bars->v_full[s]);
-        mbar_arrive_expect_tx(full, kVStage);
-        const uint32_t dst = c.base + v_stage_off(s);
+      block_rows(p, g, cur, j, c.lane, &blk);
+      for (int n = 0; n < 2; ++n, ++vit) {
+        const int s = vit % kVSlots;
+        if (!warp_wait(bar_addr(c.bars->v_empty[s]), ((vit / kVSlots) & 1u) ^ 1u, c.wc)) {
+          alive = false;
+          break;
+        }
+        if (c.lane == 0) {
+          const uint32_t full = bar_addr(c.bars->v_full[s]);
+          mbar_arrive_expect_tx(full, kVSlot);
+          const uint32_t dst = c.base + v_slot_off(s);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) tma_load_2d(dst + ch * kChunk, tmap, ch * 64, blk * kBlock, full);
+          for (int q = 0; q < 4; ++q) tma_load_2d(dst + q * kChunk, tmap, (4 * n + q) * 64, blk * kBlock, full);
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
   }
   if (!alive) {
-    for (uint32_t k = (it > kNV ? it - kNV : 0); k < it; ++k) {
+    for (uint32_t k = (vit > kVSlots ? vit - kVSlots : 0); k < vit; ++k) {
       const long long t0 = clock64();
-      while (!mbar_try_wait(bar_addr(c, c.bars->v_full[k % kNV]), (k / kNV) & 1u) &&
+      while (!mbar_try_wait(bar_addr(c.bars->v_full[k % kVSlots]), (k / kVSlots) & 1u) &&
              clock64() - t0 < 2000000000LL) {
       }
     }
   }
 }
 
-// Rows at or past the valid count of a block are zeroed in the V tile, so that
-// whatever the cache holds there (even NaN) contributes exactly 0 * 0.  This
-// warp visits every block (arriving on v_fixed even when nothing needs
-// zeroing) so that its barrier phases stay in lockstep with the stages.
+// Rows at or past the valid count of a block are zeroed in the V slots, so
+// that whatever the cache holds there (even NaN) contributes exactly 0 * 0.
+// This warp visits every slot fill (arriving on v_fixed even when nothing
+// needs zeroing) so that its barrier phases stay in lockstep with the ring.
 __device__ void value_fixup(const Ctx& c) {
   const DecodeParams& p = *c.p;
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
-  uint32_t it = 0;
+  BlockCursor cur;
+  uint32_t vit = 0;
   while (w.next(g)) {
-    for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
+    cur.reset(p, g);
+    for (int j = g.blk_lo; j < g.blk_hi; ++j) {
       int blk;
-      const int nv = block_rows(p, g, j, &blk);
-      const int s = it % kNV;
-      if (!warp_wait(bar_addr(c, c.bars->v_full[s]), (it / kNV) & 1u, c.wc)) return;
-      if (nv < kBlock) {
-        uint8_t* st = c.gbase + v_stage_off(s);
-        const int rows = kBlock - nv;
-        for (int idx = c.lane; idx < rows * 8 * 8; idx += 32) {
-          const int ch = idx / (rows * 8);
-          const int rem = idx % (rows * 8);
-          const int row = nv + rem / 8;
-          const int q16 = rem % 8;
-          *reinterpret_cast<uint4*>(st + ch * kChunk + row * 128 + q16 * 16) = make_uint4(0, 0, 0, 0);
+      const int nv = block_rows(p, g, cur, j, c.lane, &blk);
+      for (int n = 0; n < 2; ++n, ++vit) {
+        const int s = vit % kVSlots;
+        if (!warp_wait(bar_addr(c.bars->v_full[s]), (vit / kVSlots) & 1u, c.wc)) return;
+        if (nv < kBlock) {
+          uint8_t* st = c.gbase + v_slot_off(s);
+          const int rows = kBlock - nv;
+          for (int idx = c.lane; idx < rows * 4 * 8; idx += 32) {
+            const int ch = idx / (rows * 8);
+            const int rem = idx % (rows * 8);
+            const int row = nv + rem / 8;
+            const int q16 = rem % 8;
+            *reinterpret_cast<uint4*>(st + ch * kChunk + row * 128 + q16 * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        __syncwarp();
+        if (c.lane == 0) mbar_arrive(bar_addr(c.bars->v_fixed[s]));
       }
-      __syncwarp();
-      if (c.lane == 0) mbar_arrive(bar_addr(c, c.bars->v_fixed[s]));
     }
   }
 }
@@ -400,46 +594,48 @@ __device__ void value_mma(const Ctx& c) {
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
-  uint32_t it = 0, seg = 0, ncorr = 0;
+  uint32_t it = 0, vit = 0, seg = 0, ncorr = 0;
   while (w.next(g)) {
     if (seg > 0) {
-      if (!warp_wait(bar_addr(c, c.bars->o_free), (seg - 1) & 1u, c.wc)) return;
+      if (!warp_wait(bar_addr(c.bars->o_free), (seg - 1) & 1u, c.wc)) return;
       tc_fence_after();
     }
     for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
-      int blk;
-      const int nv = block_rows(p, g, j, &blk);
-      const int s = it % kNV;
       const int r = it % kNP;
-      (void)nv;
-      if (!warp_wait(bar_addr(c, c.bars->v_full[s]), (it / kNV) & 1u, c.wc)) return;
-      if (!warp_wait(bar_addr(c, c.bars->v_fixed[s]), (it / kNV) & 1u, c.wc)) return;
-      if (!warp_wait(bar_addr(c, c.bars->p_full[r]), (it / kNP) & 1u, c.wc)) return;
+      if (!warp_wait(bar_addr(c.bars->p_full[r]), (it / kNP) & 1u, c.wc)) return;
       const bool first = (j == g.blk_lo);
       const uint8_t* meta = c.gbase + meta_rec_off(r);
       uint32_t any = 0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) any |= reinterpret_cast<const uint32_t*>(meta + q * kMetaWarp)[96];
       if (any && !first) {
-        if (!warp_wait(bar_addr(c, c.bars->corr_done), ncorr & 1u, c.wc)) return;
+        // hand O over for rescaling once every MMA issued so far (the previous
+        // block's PV) has completed, and take it back when rescaled
+        if (c.lane == 0) mma_commit(bar_addr(c.bars->pv_prev));
+        __syncwarp();
+        if (!warp_wait(bar_addr(c.bars->corr_done), ncorr & 1u, c.wc)) return;
         ++ncorr;
       }
-      tc_fence_after();
-      if (c.lane == 0) {
-        const uint32_t pa = c.base + p_rec_off(r);
-        const uint32_t va = c.base + v_stage_off(s);
+      fence_proxy_async_smem();
+      const uint32_t pa = c.base + p_rec_off(r);
+      for (int n = 0; n < 2; ++n, ++vit) {
+        const int s = vit % kVSlots;
+        if (!warp_wait(bar_addr(c.bars->v_full[s]), (vit / kVSlots) & 1u, c.wc)) return;
+        if (!warp_wait(bar_addr(c.bars->v_fixed[s]), (vit / kVSlots) & 1u, c.wc)) return;
+        tc_fence_after();
+        if (c.lane == 0) {
+          const uint32_t va = c.base + v_slot_off(s);
 #pragma unroll
-        for (int k = 0; k < kBlock / 16; ++k) {
-          const uint64_t adesc = sw128_desc(pa + k * 32, 16, 1024);
-#pragma unroll
-          for (int n = 0; n < 2; ++n) {
-            const uint64_t bdesc = sw128_desc(va + n * 4 * kChunk + k * 2048, kChunk, 1024);
-            mma_ss(c.tmem + 256 * n, adesc, bdesc, kIdescPV, (k > 0 || !first) ? 1u : 0u);
-          }
+          for (int k = 0; k < kBlock / 16; ++k)
+            mma_ss(c.tmem + 256 * n, sw128_desc(pa + k * 32, 16, 1024),
+                   sw128_desc(va + k * 2048, kChunk, 1024), kIdescPV, (k > 0 || !first) ? 1u : 0u);
+          mma_commit(bar_addr(c.bars->v_empty[s]));
         }
-        mma_commit(bar_addr(c, c.bars->v_empty[s]));
-        mma_commit(bar_addr(c, c.bars->pv_done));
-        mma_commit_mc(bar_addr(c, c.bars->p_empty[r]), 0x1);
+        __syncwarp();
+      }
+      if (c.lane == 0) {
+        mma_commit_mc(bar_addr(c.bars->p_empty[r]), 0x1);
+        if (j == g.blk_hi - 1) mma_commit(bar_addr(c.bars->o_ready));  // O final for this segment
       }
       __syncwarp();
     }
@@ -455,12 +651,12 @@ __device__ void value_epilogue(const Ctx& c) {
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
-  uint32_t it = 0;
+  uint32_t it = 0, seg = 0, ncorr = 0;
   while (w.next(g)) {
     float m_fin = -INFINITY, l_fin = 0.f;
     for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
       const int r = it % kNP;
-      if (!warp_wait(bar_addr(c, c.bars->p_full[r]), (it / kNP) & 1u, c.wc)) return;
+      if (!warp_wait(bar_addr(c.bars->p_full[r]), (it / kNP) & 1u, c.wc)) return;
       const uint8_t* meta = c.gbase + meta_rec_off(r);
       const float alpha = reinterpret_cast<const float*>(meta + q4 * kMetaWarp)[c.lane];
       uint32_t any = 0;
@@ -473,10 +669,11 @@ __device__ void value_epilogue(const Ctx& c) {
         l_fin = reinterpret_cast<const float*>(meta + q4 * kMetaWarp)[64 + c.lane];
       }
       __syncwarp();
-      if (c.lane == 0) mbar_arrive_remote(bar_addr(c, c.bars->p_empty[r]), 0);
+      if (c.lane == 0) mbar_arrive_remote(bar_addr(c.bars->p_empty[r]), 0);
       if (any && !first) {
-        // O must hold the previous block's PV before it is rescaled
-        if (!warp_wait(bar_addr(c, c.bars->pv_done), (it - 1) & 1u, c.wc)) return;
+        // the MMA warp hands O over (pv_prev) once the previous block's PV is done
+        if (!warp_wait(bar_addr(c.bars->pv_prev), ncorr & 1u, c.wc)) return;
+        ++ncorr;
         tc_fence_after();
 #pragma unroll 1
         for (int ch = 0; ch < 16; ++ch) {
@@ -489,10 +686,10 @@ __device__ void value_epilogue(const Ctx& c) {
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar_addr(c, c.bars->corr_done));
+        mbar_arrive(bar_addr(c.bars->corr_done));
       }
       if (last) {
-        if (!warp_wait(bar_addr(c, c.bars->pv_done), it & 1u, c.wc)) return;
+        if (!warp_wait(bar_addr(c.bars->o_ready), seg & 1u, c.wc)) return;
         tc_fence_after();
         const bool live = h < p.H;
         const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
@@ -525,7 +722,7 @@ __device__ void value_epilogue(const Ctx& c) {
           }
         }
         tc_fence_before();
-        mbar_arrive(bar_addr(c, c.bars->o_free));
+        mbar_arrive(bar_addr(c.bars->o_free));
         if (live) {
           if (g.slot < 0)
             p.lse[size_t(g.b) * p.H + h] = lse;
@@ -535,6 +732,7 @@ __device__ void value_epilogue(const Ctx& c) {
         if (h == 0 && g.first_of_seq) p.seq_info[g.b] = seq_info_for(g, w);
       }
     }
+    ++seg;
   }
 }
 
@@ -552,7 +750,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kNK; ++s) {
+    for (int s = 0; s < kKSlots; ++s) {
       mbar_init(smem_u32(&bars->k_full[s]), 1);
       mbar_init(smem_u32(&bars->k_empty[s]), 1);
     }
@@ -564,15 +762,18 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
     mbar_init(smem_u32(&bars->q_free), 1);
     for (int r = 0; r < kNP; ++r) {
       mbar_init(smem_u32(&bars->p_empty[r]), 1 + 4);  // PV commit + 4 epilogue warps
-      mbar_init(smem_u32(&bars->p_full[r]), 4);       // 4 softmax warps (expect_tx each)
+      mbar_init(smem_u32(&bars->p_full[r]), 64);      // every sender thread (+ st.async bytes)
+      mbar_init(smem_u32(&bars->stage_full[r]), 128); // every softmax thread
+      mbar_init(smem_u32(&bars->stage_empty[r]), 64); // every sender thread
     }
-    for (int s = 0; s < kNV; ++s) {
+    for (int s = 0; s < kVSlots; ++s) {
       mbar_init(smem_u32(&bars->v_full[s]), 1);
       mbar_init(smem_u32(&bars->v_empty[s]), 1);
       mbar_init(smem_u32(&bars->v_fixed[s]), 1);
     }
-    mbar_init(smem_u32(&bars->pv_done), 1);
+    mbar_init(smem_u32(&bars->pv_prev), 1);
     mbar_init(smem_u32(&bars->corr_done), 128);
+    mbar_init(smem_u32(&bars->o_ready), 1);
     mbar_init(smem_u32(&bars->o_free), 128);
     bars->abort = 0;
     fence_mbar_init();
@@ -599,7 +800,8 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
   if (rank == 0) {
     if (warp == 0) score_tma(c, &tmap);
     else if (warp == 1) score_mma(c);
-    else if (warp >= 4) score_softmax(c);
+    else if (warp <= 3) score_sender(c);
+    else score_softmax(c);
   } else {
     if (warp == 0) value_tma(c, &tmap);
     else if (warp == 1) value_mma(c);
@@ -628,12 +830,15 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
 size_t decode_sm100_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(kSmemBytes));
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev] = true;
   }
   decode_sm100_kernel<<<dim3(2 * p.P), kThreads, kSmemBytes, stream>>>(tmap, p);
   return cudaGetLastError();
