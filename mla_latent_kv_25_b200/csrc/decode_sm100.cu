@@ -43,20 +43,22 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 256;
-constexpr int kKSlots = 9;   // score CTA: ring of [128 tokens x 64 cols] chunk slots
+constexpr int kKChunks = 3;  // score CTA: 64-column chunks per K slot
+constexpr int kKSlots = 3;   // score CTA: ring of [128 tokens x 192 cols] slots (one pass = 3 slots)
 constexpr int kVSlots = 5;   // value CTA: ring of [64 tokens x 256 cols] half-block slots
 constexpr int kNP = 3;       // P records in flight
 constexpr int kNS = 2;       // S accumulators (128 columns each) in TMEM
 
 constexpr uint32_t kChunk = 64 * 128;          // one [64 rows x 64 bf16] swizzled chunk
-constexpr uint32_t kKSlot = 2 * kChunk;         // [128 rows x 64 bf16]
+constexpr uint32_t kKPair = 2 * kChunk;         // one chunk of both blocks: [128 rows x 64 bf16]
+constexpr uint32_t kKSlot = kKChunks * kKPair;   // [128 rows x 192 bf16] as 3 swizzled [128 x 64] tiles
+static_assert(9 % kKChunks == 0, "a pass is a whole number of K slots");
 constexpr uint32_t kVSlot = 4 * kChunk;         // [64 rows x 256 bf16]
 constexpr uint32_t kPBytes = 128 * 64 * 2;     // P [128 heads x 64 tokens] bf16
 constexpr uint32_t kQRopeBytes = 128 * 64 * 2; // RoPE part of Q [128 heads x 64] bf16
 constexpr uint32_t kMetaWarp = 400;            // per warp: alpha[32] m[32] l[32] flag + pad
 constexpr uint32_t kMetaBytes = 4 * kMetaWarp;
 constexpr float kRescaleThreshold = 8.0f;      // log2 units
-constexpr int kPrefetchAhead = 8;              // blocks prefetched into L2 ahead of the K ring
 constexpr float kLog2e = 1.4426950408889634f;
 
 // TMEM columns of the score CTA: latent part of Q (512 bf16 = 256 columns), then S.
@@ -165,28 +167,9 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   uint32_t cit = 0;
   bool alive = true;
   if (c.lane == 0) prefetch_tmap(tmap);
-  const uint8_t* cache = static_cast<const uint8_t*>(p.cache);
-  BlockCursor pcur;  // block ids for the L2 prefetch, kPrefetchAhead blocks ahead
   while (alive && w.next(g)) {
     cur.reset(p, g);
-    pcur.reset(p, g);
-    // warm L2 with the first blocks of the segment; from then on each pass
-    // prefetches the two blocks kPrefetchAhead ahead, so the ring's TMA loads
-    // hit L2 (the ring itself is too small to cover HBM latency)
-    for (int j = g.blk_lo; j < g.blk_lo + kPrefetchAhead && j < g.blk_hi; ++j) {
-      int pb;
-      const int nv = block_rows(p, g, pcur, j, c.lane, &pb);
-      if (c.lane == 0 && nv > 0) prefetch_l2_bulk(cache + size_t(pb) * kBlock * kRow * 2, kBlock * kRow * 2);
-    }
     for (int j = g.blk_lo; alive && j < g.blk_hi; j += 2) {
-      for (int q = 0; q < 2; ++q) {
-        const int jp = j + kPrefetchAhead + q;
-        if (jp < g.blk_hi) {
-          int pb;
-          const int nv = block_rows(p, g, pcur, jp, c.lane, &pb);
-          if (c.lane == 0 && nv > 0) prefetch_l2_bulk(cache + size_t(pb) * kBlock * kRow * 2, kBlock * kRow * 2);
-        }
-      }
       int blk_a, blk_b = 0;
       const int nv_a = block_rows(p, g, cur, j, c.lane, &blk_a);
       const bool has_b = j + 1 < g.blk_hi;
@@ -196,7 +179,10 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
         if (nv_a == 0 && g.len > j * kBlock) atomicOr(p.err, kErrBadBlock);
         if (has_b && nv_b == 0) atomicOr(p.err, kErrBadBlock);
       }
-      for (int ch = 0; ch < 9; ++ch, ++cit) {
+      // one K slot = kKChunks column chunks of both blocks: few, large TMA
+      // transactions per barrier (per-SM TMA throughput grows with the bytes
+      // one barrier tracks)
+      for (int i = 0; i < 9 / kKChunks; ++i, ++cit) {
         const int s = cit % kKSlots;
         if (!warp_wait(bar_addr(c.bars->k_empty[s]), ((cit / kKSlots) & 1u) ^ 1u, c.wc)) {
           alive = false;
@@ -204,10 +190,14 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
         }
         if (c.lane == 0) {
           const uint32_t full = bar_addr(c.bars->k_full[s]);
-          mbar_arrive_expect_tx(full, has_b ? kKSlot : kChunk);
+          mbar_arrive_expect_tx(full, (has_b ? 2u : 1u) * kKChunks * kChunk);
           const uint32_t dst = c.base + k_slot_off(s);
-          tma_load_2d(dst, tmap, ch * 64, blk_a * kBlock, full);
-          if (has_b) tma_load_2d(dst + kChunk, tmap, ch * 64, blk_b * kBlock, full);
+#pragma unroll
+          for (int q = 0; q < kKChunks; ++q) {
+            const int ch = i * kKChunks + q;
+            tma_load_2d(dst + q * kKPair, tmap, ch * 64, blk_a * kBlock, full);
+            if (has_b) tma_load_2d(dst + q * kKPair + kChunk, tmap, ch * 64, blk_b * kBlock, full);
+          }
         }
         __syncwarp();
       }
@@ -217,7 +207,7 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   if (!alive) {
     for (uint32_t k = (cit > kKSlots ? cit - kKSlots : 0); k < cit; ++k) {
       const long long t0 = clock64();
-      while (!mbar_try_wait(bar_addr(c.bars->k_full[k % kKSlots]), (k / kKSlots) & 1u) &&
+      while (!mbar_test_wait(bar_addr(c.bars->k_full[k % kKSlots]), (k / kKSlots) & 1u) &&
              clock64() - t0 < 2000000000LL) {
       }
     }
@@ -238,19 +228,23 @@ __device__ void score_mma(const Ctx& c) {
       const int sb = pit % kNS;
       if (!warp_wait(bar_addr(c.bars->s_empty[sb]), ((pit / kNS) & 1u) ^ 1u, c.wc)) return;
       const uint32_t d = c.tmem + kSCol + sb * 128;
-      for (int ch = 0; ch < 9; ++ch, ++cit) {
+      for (int i = 0; i < 9 / kKChunks; ++i, ++cit) {
         const int s = cit % kKSlots;
         if (!warp_wait(bar_addr(c.bars->k_full[s]), (cit / kKSlots) & 1u, c.wc)) return;
         tc_fence_after();
         if (c.lane == 0) {
-          const uint32_t slot = c.base + k_slot_off(s);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t b = sw128_desc(slot + kk * 32, 16, 1024);
-            if (ch < 8)
-              mma_ts(d, c.tmem + kQCol + 32 * ch + 8 * kk, b, kIdescQK, (ch | kk) ? 1u : 0u);
-            else
-              mma_ss(d, sw128_desc(qrope + kk * 32, 16, 1024), b, kIdescQK, 1u);
+          for (int q = 0; q < kKChunks; ++q) {
+            const int ch = i * kKChunks + q;
+            const uint32_t tile = c.base + k_slot_off(s) + q * kKPair;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t b = sw128_desc(tile + kk * 32, 16, 1024);
+              if (ch < 8)
+                mma_ts(d, c.tmem + kQCol + 32 * ch + 8 * kk, b, kIdescQK, (ch | kk) ? 1u : 0u);
+              else
+                mma_ss(d, sw128_desc(qrope + kk * 32, 16, 1024), b, kIdescQK, 1u);
+            }
           }
           mma_commit(bar_addr(c.bars->k_empty[s]));
         }
@@ -544,7 +538,7 @@ __device__ void value_tma(const Ctx& c, const CUtensorMap* tmap) {
   if (!alive) {
     for (uint32_t k = (vit > kVSlots ? vit - kVSlots : 0); k < vit; ++k) {
       const long long t0 = clock64();
-      while (!mbar_try_wait(bar_addr(c.bars->v_full[k % kVSlots]), (k / kVSlots) & 1u) &&
+      while (!mbar_test_wait(bar_addr(c.bars->v_full[k % kVSlots]), (k / kVSlots) & 1u) &&
              clock64() - t0 < 2000000000LL) {
       }
     }
