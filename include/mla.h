@@ -69,10 +69,19 @@ typedef enum {
  * q_nope: bf16 [B,H,128]; w_uk: bf16 [H,128,512]; q_rope: bf16 [B,H,64] or NULL;
  * q_out: bf16 rows of stride ldq elements (ldq >= 512, >= 576 if q_rope != NULL,
  * a multiple of 8; 576 builds the packed [B,H,576] query mla_decode reads).
- * fp32 accumulation, one bf16 rounding.  B >= 1.  All pointers 16-byte aligned.
+ * fp32 accumulation (tensor cores), one bf16 rounding.  B >= 1.  All pointers
+ * 16-byte aligned; q_nope and w_uk dense in the layouts above.
  */
 mla_status_t mla_absorb_q(const void *q_nope, const void *w_uk, const void *q_rope,
                           void *q_out, int ldq, int B, int H, void *stream);
+
+/*
+ * mla_absorb_get_error - device error bits of the mla_absorb_q launches since
+ * the last call (MLA_DEVERR_TIMEOUT when a bounded wait in the kernel gave up;
+ * the affected rows are then not written).  Synchronises `stream` and clears
+ * the bits.  MLA_ERR_INVALID_ARG if err_bits is NULL.
+ */
+mla_status_t mla_absorb_get_error(void *stream, uint32_t *err_bits);
 
 /*
  * mla_decode_workspace_bytes - bytes of device workspace mla_decode needs for
@@ -160,7 +169,7 @@ mla_status_t mla_get_device_error(void *workspace, void *stream, uint32_t *err_b
  * loads the library until the process exits.  A request whose scratch need
  * (mla_decode_workspace_bytes(B, H, num_splits)) exceeds 40 MiB returns
  * MLA_ERR_WORKSPACE_TOO_SMALL and launches nothing (at H = 128 the automatic
- * split count of a B200 needs about 39 MB).  The first call on a device looks
+ * split count of a B200 needs at most about 39 MB).  The first call on a device looks
  * up the array's address on that device; make it before any stream capture.
  * All calls on a device share the array and it keeps the last call's
  * contents: calls that overlap on the GPU race, so serialise them.  Nothing

@@ -29,8 +29,9 @@ DEVERR_SEQ_TOO_LONG = 0x2
 DEVERR_TIMEOUT = 0x4
 
 # every symbol include/mla.h declares
-EXPORTS = ("mla_absorb_q", "mla_decode_workspace_bytes", "mla_decode", "mla_combine",
-           "mla_get_device_error", "mla_status_string", "mla_num_sms", "mla_decode_noalloc")
+EXPORTS = ("mla_absorb_q", "mla_absorb_get_error", "mla_decode_workspace_bytes", "mla_decode",
+           "mla_combine", "mla_get_device_error", "mla_status_string", "mla_num_sms",
+           "mla_decode_noalloc")
 
 
 class MLAError(RuntimeError):
@@ -56,6 +57,8 @@ def load():
         vp, i32, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         L.mla_absorb_q.restype = i32
         L.mla_absorb_q.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
+        L.mla_absorb_get_error.restype = i32
+        L.mla_absorb_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_decode_workspace_bytes.restype = u64
         L.mla_decode_workspace_bytes.argtypes = [i32, i32, i32]
         L.mla_decode.restype = i32
@@ -138,6 +141,13 @@ def mla_absorb_q(q_nope, w_uk, q_rope, q_out, stream=None):
     _check("mla_absorb_q", load().mla_absorb_q(_ptr(q_nope), _ptr(w_uk), _ptr(q_rope), _ptr(q_out),
                                                ldq, B, H, _stream(stream)))
     return q_out
+
+
+def mla_absorb_get_error(stream=None) -> int:
+    """Synchronise the stream, return and clear the absorption kernel's error bits."""
+    v = ctypes.c_uint32(0)
+    _check("mla_absorb_get_error", load().mla_absorb_get_error(_stream(stream), ctypes.byref(v)))
+    return int(v.value)
 
 
 def mla_decode(q, cache, block_table, seq_lens, softmax_scale, out, lse, workspace, *,

@@ -1,63 +1,180 @@
-// Query absorption: q_out[b,h,0:512] = q_nope[b,h,:] . W_UK[h]  (K = 128),
-// q_out[b,h,512:576] = q_rope[b,h,:].  One CTA per (head, 16 batch rows);
-// thread t owns latent columns 2t, 2t+1; fp32 accumulation, one bf16 rounding.
+// Query absorption on tcgen05 tensor cores:
+//   q_out[b,h,0:512]   = q_nope[b,h,:] . W_UK[h]      (K = 128, fp32 accumulation, one bf16 rounding)
+//   q_out[b,h,512:576] = q_rope[b,h,:]                (copied)
+//
+// One CTA per (head h, tile of 128 batch rows).  Per head this is a plain GEMM
+// D[128 x 512] = A[128 x 128] . B[128 x 512] with
+//   A = q_nope rows of head h (K-major, rows past B read as zeros by TMA),
+//   B = W_UK[h] stored [d][c] (c contiguous, so MN-major),
+//   D = fp32 in all 512 TMEM columns.
+// The operands are staged by TMA in two K halves (one barrier each) so the
+// MMAs of the first half overlap the second half's load; 16 MMAs of
+// 128 x 256 x 16 in total.  The epilogue: each of the 4 warps reads its 32
+// TMEM lanes (= 32 batch rows) and writes bf16 rows.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace mla {
 
+// Error word of the absorption kernel (the call has no workspace): bit
+// kErrTimeout when a bounded wait gave up.  Read and cleared by
+// mla_absorb_get_error.
+__device__ uint32_t g_absorb_err;
+
 namespace {
 
-constexpr int kRowsPerCta = 16;
-constexpr int kThreads = 256;
+using namespace sm100;
 
-__global__ void __launch_bounds__(kThreads)
-absorb_q_kernel(const __nv_bfloat16* __restrict__ q_nope, const __nv_bfloat16* __restrict__ w_uk,
-                const __nv_bfloat16* __restrict__ q_rope, __nv_bfloat16* __restrict__ q_out,
-                int ldq, int B, int H) {
-  __shared__ float qs[kRowsPerCta][kNope];
+constexpr int kThreads = 128;
+constexpr uint32_t kATile = 128 * 128;        // [128 rows x 64 d] bf16, swizzled
+constexpr uint32_t kWBox = 64 * 128;          // [64 d x 64 c] bf16
+constexpr uint32_t kWChunk = 2 * kWBox;       // [128 d x 64 c]: one 64-column chunk of W_UK[h]
+constexpr uint32_t kAOff = 1024;              // after the barrier block
+constexpr uint32_t kWOff = kAOff + 2 * kATile;
+constexpr uint32_t kSmem = kWOff + 8 * kWChunk + 1024;
+static_assert(kSmem <= 232448, "shared memory budget");
+constexpr uint32_t kHalfBytes = kATile + 8 * kWBox;  // A tile + 8 W boxes per K half
+constexpr uint32_t kIdesc = idesc_bf16(128, 256, false, true);
+
+struct Bars {
+  uint64_t full[2];
+  uint64_t done;
+  uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+absorb_sm100_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap wmap,
+                    const __nv_bfloat16* __restrict__ q_rope, __nv_bfloat16* __restrict__ q_out,
+                    int ldq, int B, int H, long long spin_limit) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  Bars* bars = reinterpret_cast<Bars*>(smem_raw + (base - raw));
   const int h = blockIdx.x;
-  const int b0 = blockIdx.y * kRowsPerCta;
-  const int nb = min(kRowsPerCta, B - b0);
-  const int tid = threadIdx.x;
-  for (int i = tid; i < kRowsPerCta * kNope; i += kThreads) {
-    int r = i / kNope, d = i % kNope;
-    qs[r][d] = r < nb ? __bfloat162float(q_nope[(size_t(b0 + r) * H + h) * kNope + d]) : 0.f;
+  const int b0 = blockIdx.y * 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->full[0]), 1);
+    mbar_init(smem_u32(&bars->full[1]), 1);
+    mbar_init(smem_u32(&bars->done), 1);
+    abort_flag = 0;
+    fence_mbar_init();
   }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  float acc[kRowsPerCta][2];
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const WaitCtx wc{spin_limit, &g_absorb_err, &abort_flag};
+
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&qmap);
+    prefetch_tmap(&wmap);
+    for (int kc = 0; kc < 2; ++kc) {
+      const uint32_t full = smem_u32(&bars->full[kc]);
+      mbar_arrive_expect_tx(full, kHalfBytes);
+      // A: d in [64 kc, 64 kc + 64), rows b0..b0+127 of head h
+      asm volatile(
+          "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+          " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(base + kAOff + kc * kATile),
+          "l"(reinterpret_cast<uint64_t>(&qmap)), "r"(64 * kc), "r"(h), "r"(b0), "r"(full)
+          : "memory");
+      // W_UK[h] rows d in the same half, all 8 column chunks
+      for (int j = 0; j < 8; ++j)
+        tma_load_2d(base + kWOff + j * kWChunk + kc * kWBox, &wmap, 64 * j, h * 128 + 64 * kc, full);
+    }
+    for (int kc = 0; kc < 2; ++kc) {
+      if (!wait_phase(smem_u32(&bars->full[kc]), 0, wc)) break;
+      tc_fence_after();
 #pragma unroll
-  for (int r = 0; r < kRowsPerCta; ++r) acc[r][0] = acc[r][1] = 0.f;
-  const __nv_bfloat162* w = reinterpret_cast<const __nv_bfloat162*>(w_uk + size_t(h) * kNope * kDc);
-#pragma unroll 4
-  for (int d = 0; d < kNope; ++d) {
-    float2 wv = __bfloat1622float2(w[size_t(d) * (kDc / 2) + tid]);
+      for (int kk = 0; kk < 4; ++kk) {
+        const int k = 4 * kc + kk;  // 16-wide step along d
+        const uint64_t a = sw128_desc(base + kAOff + kc * kATile + kk * 32, 16, 1024);
 #pragma unroll
-    for (int r = 0; r < kRowsPerCta; ++r) {
-      float a = qs[r][d];
-      acc[r][0] += a * wv.x;
-      acc[r][1] += a * wv.y;
+        for (int n = 0; n < 2; ++n) {
+          const uint64_t b = sw128_desc(base + kWOff + 4 * n * kWChunk + k * 2048, kWChunk, 1024);
+          mma_ss(tmem + 256 * n, a, b, kIdesc, k > 0 ? 1u : 0u);
+        }
+      }
+    }
+    mma_commit(smem_u32(&bars->done));
+  }
+  __syncwarp();
+  const bool ok = warp_wait(smem_u32(&bars->done), 0, wc) && !*static_cast<volatile int*>(&abort_flag);
+  tc_fence_after();
+
+  const int row = warp * 32 + lane;
+  const int b = b0 + row;
+  const bool live = ok && b < B;
+  __nv_bfloat16* dst = q_out + (size_t(b) * H + h) * ldq;
+#pragma unroll 1
+  for (int ch = 0; ch < 16; ++ch) {
+    uint32_t v[32];
+    tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 32 * ch, v);
+    tmem_ld_wait();
+    if (!live) continue;
+    uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]),
+                                                  __uint_as_float(v[8 * q + 2 * e + 1]));
+        w4[e] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      d4[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
   }
-  for (int r = 0; r < nb; ++r) {
-    __nv_bfloat16* dst = q_out + (size_t(b0 + r) * H + h) * ldq;
-    reinterpret_cast<__nv_bfloat162*>(dst)[tid] = __floats2bfloat162_rn(acc[r][0], acc[r][1]);
-    if (q_rope != nullptr && tid < kDr / 2) {
-      const __nv_bfloat162* src =
-          reinterpret_cast<const __nv_bfloat162*>(q_rope + (size_t(b0 + r) * H + h) * kDr);
-      reinterpret_cast<__nv_bfloat162*>(dst + kDc)[tid] = src[tid];
-    }
+  if (live && q_rope != nullptr) {
+    const uint4* src = reinterpret_cast<const uint4*>(q_rope + (size_t(b) * H + h) * kDr);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + kDc);
+#pragma unroll
+    for (int q = 0; q < kDr / 8; ++q) d4[q] = src[q];
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace
 
-cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* w_uk,
+cudaError_t launch_absorb_q(const CUtensorMap& qmap, const CUtensorMap& wmap,
                             const __nv_bfloat16* q_rope, __nv_bfloat16* q_out, int ldq, int B,
-                            int H, cudaStream_t stream) {
-  dim3 grid(H, (B + kRowsPerCta - 1) / kRowsPerCta);
-  absorb_q_kernel<<<grid, kThreads, 0, stream>>>(q_nope, w_uk, q_rope, q_out, ldq, B, H);
+                            int H, long long spin_limit, cudaStream_t stream) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(absorb_sm100_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid(H, (B + 127) / 128);
+  absorb_sm100_kernel<<<grid, kThreads, kSmem, stream>>>(qmap, wmap, q_rope, q_out, ldq, B, H,
+                                                         spin_limit);
   return cudaGetLastError();
+}
+
+cudaError_t absorb_take_error(uint32_t* bits, cudaStream_t stream) {
+  uint32_t* dev = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&dev), g_absorb_err);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemcpyAsync(bits, dev, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
+    return e;
+  if ((e = cudaMemsetAsync(dev, 0, sizeof(uint32_t), stream)) != cudaSuccess) return e;
+  return cudaStreamSynchronize(stream);
 }
 
 }  // namespace mla

@@ -41,15 +41,19 @@ int device_max_clusters() {
   return cache[dev];
 }
 
-// Engines of the split-KV partition: by default one per co-resident cluster
-// of two SMs.
-int resolve_engines(int num_splits) {
+// Engines of the split-KV partition.  By default one per co-resident cluster
+// of two SMs; but when the batch is at least three quarters of that and the
+// sequences are of similar length, one engine per sequence is faster: no
+// sequence is cut (no partial results, no merge) and every engine runs a
+// single segment, which outweighs the idle clusters.
+int resolve_engines(int num_splits, int B) {
   if (num_splits > 0) return num_splits;
   int sms = device_sms();
   if (sms < 2) return 0;
   int P = sms / 2;
   int mc = device_max_clusters();
   if (mc > 0 && mc < P) P = mc;
+  if (B <= P && 4 * B >= 3 * P) P = B;
   return P;
 }
 
@@ -67,19 +71,26 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D view [rows, cols] of a row-major bf16 matrix, 64 x 64 box, 128 B swizzle.
-bool encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                     uint64_t row_bytes) {
+// bf16 tensor map with 128 B swizzle: dims[0] is the contiguous dimension,
+// strides[i] the byte stride of dims[i + 1]; out-of-range reads give zeros.
+bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {64, 64};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// 2-D view [rows, cols] of a row-major bf16 matrix, 64 x 64 box.
+bool encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                     uint64_t row_bytes) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {64, 64};
+  return encode_bf16(map, base, 2, dims, strides, box);
 }
 
 constexpr int kMaxSplits = 4096;
@@ -109,7 +120,7 @@ int mla_num_sms(void) { return device_sms(); }
 size_t mla_decode_workspace_bytes(int B, int H, int num_splits) {
   if (B < 1 || B > kMaxBatch || !valid_heads(H) || num_splits < 0 || num_splits > kMaxSplits)
     return 0;
-  int P = resolve_engines(num_splits);
+  int P = resolve_engines(num_splits, B);
   if (P < 1) return 0;
   return ws_layout(B, H, P).total;
 }
@@ -121,12 +132,26 @@ mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, const void* q_ro
   if (ldq < (q_rope ? kRow : kDc) || ldq % 8 != 0) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_nope) || !aligned16(w_uk) || !aligned16(q_out) || (q_rope && !aligned16(q_rope)))
     return MLA_ERR_INVALID_ARG;
-  cudaError_t e = launch_absorb_q(static_cast<const __nv_bfloat16*>(q_nope),
-                                  static_cast<const __nv_bfloat16*>(w_uk),
-                                  static_cast<const __nv_bfloat16*>(q_rope),
-                                  static_cast<__nv_bfloat16*>(q_out), ldq, B, H,
+  // q_nope [B, H, 128] as {d, h, b}: one box = 128 batch rows x 64 d of one head
+  CUtensorMap qmap, wmap;
+  const cuuint64_t qdims[3] = {cuuint64_t(kNope), cuuint64_t(H), cuuint64_t(B)};
+  const cuuint64_t qstr[2] = {cuuint64_t(kNope) * 2, cuuint64_t(H) * kNope * 2};
+  const cuuint32_t qbox[3] = {64, 1, 128};
+  if (!encode_bf16(&qmap, q_nope, 3, qdims, qstr, qbox)) return MLA_ERR_CUDA;
+  // W_UK [H, 128, 512] as rows (h, d) x columns c
+  if (!encode_bf16_map(&wmap, w_uk, uint64_t(H) * kNope, kDc, kDc * 2)) return MLA_ERR_CUDA;
+  cudaError_t e = launch_absorb_q(qmap, wmap, static_cast<const __nv_bfloat16*>(q_rope),
+                                  static_cast<__nv_bfloat16*>(q_out), ldq, B, H, kDefaultSpin,
                                   static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_absorb_get_error(void* stream, uint32_t* err_bits) {
+  if (!err_bits) return MLA_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  if (absorb_take_error(&v, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  *err_bits = v;
+  return MLA_OK;
 }
 
 mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void* cache,
@@ -151,7 +176,7 @@ mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0 ||
       (block_scale && (reinterpret_cast<uintptr_t>(block_scale) & 3u) != 0))
     return MLA_ERR_INVALID_ARG;
-  const int P = resolve_engines(num_splits);
+  const int P = resolve_engines(num_splits, B);
   if (P < 1) return MLA_ERR_CUDA;
   const WsLayout ws = ws_layout(B, H, P);
   if (workspace_bytes < ws.total) return MLA_ERR_WORKSPACE_TOO_SMALL;

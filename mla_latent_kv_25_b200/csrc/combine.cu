@@ -18,84 +18,96 @@ namespace mla {
 
 namespace {
 
-constexpr int kMergeThreads = 128;  // 4 columns per thread
+constexpr int kRowsPerCta = 8;                  // one warp per (b,h) row
+constexpr int kMergeThreads = 32 * kRowsPerCta;
 
-// Merge n pieces of one (b,h) row.  lse_at(i) / o_at(i) give piece i.
-// Every thread of the block calls it; thread t owns columns 4t..4t+3.
+// Merge n pieces of one (b,h) row; called by one whole warp, lane l owns
+// columns 16l..16l+15.  lse_at(i) / o_at(i) give piece i.
 template <class LseAt, class OAt>
 __device__ __forceinline__ void merge_row(int n, LseAt lse_at, OAt o_at, __nv_bfloat16* out_row,
-                                          float* lse_out) {
+                                          float* lse_out, int lane) {
   float M = -INFINITY;
   for (int i = 0; i < n; ++i) M = fmaxf(M, lse_at(i));
-  const int c = threadIdx.x * 4;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int c = lane * 16;
+  float acc[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) acc[k] = 0.f;
   float L = -INFINITY;
   if (M != -INFINITY) {
     float sum = 0.f;
     for (int i = 0; i < n; ++i) sum += expf(lse_at(i) - M);
     L = M + logf(sum);
     for (int i = 0; i < n; ++i) {
-      float li = lse_at(i);
+      const float li = lse_at(i);
       if (li == -INFINITY) continue;
-      float w = expf(li - L);
-      float4 v = *reinterpret_cast<const float4*>(o_at(i) + c);
-      acc.x += w * v.x;
-      acc.y += w * v.y;
-      acc.z += w * v.z;
-      acc.w += w * v.w;
+      const float w = expf(li - L);
+      const float4* src = reinterpret_cast<const float4*>(o_at(i) + c);
+      float4 v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[q] = src[q];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[4 * q] += w * v[q].x;
+        acc[4 * q + 1] += w * v[q].y;
+        acc[4 * q + 2] += w * v[q].z;
+        acc[4 * q + 3] += w * v[q].w;
+      }
     }
   }
-  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-  uint2 pk;
-  pk.x = *reinterpret_cast<uint32_t*>(&lo);
-  pk.y = *reinterpret_cast<uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(out_row + c) = pk;
-  if (threadIdx.x == 0) *lse_out = L;
+  uint32_t pk[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * k], acc[2 * k + 1]);
+    pk[k] = *reinterpret_cast<uint32_t*>(&b2);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(out_row + c);
+  dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  if (lane == 0) *lse_out = L;
 }
 
-// grid (B, ceil(H / heads_per_cta)), 128 threads.
+// grid (B, ceil(H / kRowsPerCta)); warp w merges head blockIdx.y * kRowsPerCta + w.
 __global__ void __launch_bounds__(kMergeThreads)
 merge_pieces_kernel(const int32_t* __restrict__ seq_lens, int max_blocks, int H,
                     const int4* __restrict__ seq_info, const float* __restrict__ lse_part,
                     const float* __restrict__ o_part, __nv_bfloat16* __restrict__ out,
-                    float* __restrict__ lse, uint32_t* __restrict__ err, int heads_per_cta) {
+                    float* __restrict__ lse, uint32_t* __restrict__ err) {
   const int b = blockIdx.x;
-  const int h0 = blockIdx.y * heads_per_cta;
-  const int h1 = min(H, h0 + heads_per_cta);
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.y * kRowsPerCta + (threadIdx.x >> 5);
   int L = seq_lens[b];
   if (L < 0 || L > max_blocks * kBlock) {
     if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(err, kErrSeqTooLong);
     L = L < 0 ? 0 : max_blocks * kBlock;
   }
+  if (h >= H) return;
+  __nv_bfloat16* row = out + (size_t(b) * H + h) * kDc;
   if (L == 0) {
-    for (int h = h0; h < h1; ++h) {
-      __nv_bfloat16* row = out + (size_t(b) * H + h) * kDc;
-      *reinterpret_cast<uint2*>(row + threadIdx.x * 4) = make_uint2(0u, 0u);
-      if (threadIdx.x == 0) lse[size_t(b) * H + h] = -INFINITY;
-    }
+    uint4* dst = reinterpret_cast<uint4*>(row + lane * 16);
+    dst[0] = make_uint4(0u, 0u, 0u, 0u);
+    dst[1] = make_uint4(0u, 0u, 0u, 0u);
+    if (lane == 0) lse[size_t(b) * H + h] = -INFINITY;
     return;
   }
   const int4 info = seq_info[b];
   if (info.w != kSeqCut) return;  // written directly by its engine
   const int p0 = info.x, p1 = info.y, slot0 = info.z;
   const int n = p1 - p0 + 1;
-  for (int h = h0; h < h1; ++h) {
-    auto slot_of = [&](int i) { return i == 0 ? slot0 : 2 * (p0 + i); };
-    auto lse_at = [&](int i) { return lse_part[size_t(slot_of(i)) * H + h]; };
-    auto o_at = [&](int i) { return o_part + (size_t(slot_of(i)) * H + h) * kDc; };
-    merge_row(n, lse_at, o_at, out + (size_t(b) * H + h) * kDc, lse + size_t(b) * H + h);
-  }
+  auto slot_of = [&](int i) { return i == 0 ? slot0 : 2 * (p0 + i); };
+  auto lse_at = [&](int i) { return lse_part[size_t(slot_of(i)) * H + h]; };
+  auto o_at = [&](int i) { return o_part + (size_t(slot_of(i)) * H + h) * kDc; };
+  merge_row(n, lse_at, o_at, row, lse + size_t(b) * H + h, lane);
 }
 
-// Public combine: o_part [B,H,S,512], lse_part [B,H,S].  grid (B*H), 128 threads.
+// Public combine: o_part [B,H,S,512], lse_part [B,H,S].  grid ceil(B*H / kRowsPerCta).
 __global__ void __launch_bounds__(kMergeThreads)
-combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part, int S,
-               __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  const size_t r = blockIdx.x;
+combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part, size_t rows,
+               int S, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  const size_t r = size_t(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
+  if (r >= rows) return;
   auto lse_at = [&](int i) { return lse_part[r * S + i]; };
   auto o_at = [&](int i) { return o_part + (r * S + i) * kDc; };
-  merge_row(S, lse_at, o_at, out + r * kDc, lse + r);
+  merge_row(S, lse_at, o_at, out + r * kDc, lse + r, threadIdx.x & 31);
 }
 
 }  // namespace
@@ -104,17 +116,17 @@ cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, 
                                 const int4* seq_info, const float* lse_part, const float* o_part,
                                 __nv_bfloat16* out, float* lse, uint32_t* err,
                                 cudaStream_t stream) {
-  const int hpc = 8;
-  dim3 grid(B, (H + hpc - 1) / hpc);
+  dim3 grid(B, (H + kRowsPerCta - 1) / kRowsPerCta);
   merge_pieces_kernel<<<grid, kMergeThreads, 0, stream>>>(seq_lens, max_blocks, H, seq_info,
-                                                          lse_part, o_part, out, lse, err, hpc);
+                                                          lse_part, o_part, out, lse, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int B, int H, int S,
                            __nv_bfloat16* out, float* lse, cudaStream_t stream) {
-  combine_kernel<<<dim3(unsigned(B) * unsigned(H)), kMergeThreads, 0, stream>>>(o_part, lse_part,
-                                                                              S, out, lse);
+  const size_t rows = size_t(B) * size_t(H);
+  combine_kernel<<<dim3(unsigned((rows + kRowsPerCta - 1) / kRowsPerCta)), kMergeThreads, 0, stream>>>(
+      o_part, lse_part, rows, S, out, lse);
   return cudaGetLastError();
 }
 

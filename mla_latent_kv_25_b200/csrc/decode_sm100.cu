@@ -312,19 +312,13 @@ struct SoftmaxState {
 __device__ __forceinline__ bool softmax_block(const Ctx& c, const uint32_t (&sv)[64], int nv, bool first,
                                               float sl2, bool pos, SoftmaxState& st, uint32_t it,
                                               int h, int q4) {
-  // block max of the scaled scores (the sign of the scale decides max or min)
-  float mr;
-  if (nv == kBlock) {
-    mr = __uint_as_float(sv[0]);
+  // block max of the scaled scores: max of s * sg with sg = sign(scale), so a
+  // negative scale needs no second code path; rows at or past nv are masked
+  const float sg = pos ? 1.f : -1.f;
+  float mr = -INFINITY;
 #pragma unroll
-    for (int t = 1; t < 64; ++t) mr = pos ? fmaxf(mr, __uint_as_float(sv[t])) : fminf(mr, __uint_as_float(sv[t]));
-  } else {
-    mr = pos ? -INFINITY : INFINITY;
-#pragma unroll
-    for (int t = 0; t < 64; ++t)
-      if (t < nv) mr = pos ? fmaxf(mr, __uint_as_float(sv[t])) : fminf(mr, __uint_as_float(sv[t]));
-  }
-  const float mx = nv > 0 ? mr * sl2 : -INFINITY;
+  for (int t = 0; t < 64; ++t) mr = fmaxf(mr, t < nv ? __uint_as_float(sv[t]) * sg : -INFINITY);
+  const float mx = nv > 0 ? mr * sg * sl2 : -INFINITY;
   float alpha = 1.f;
   bool resc = false;
   if (first) {
@@ -338,24 +332,15 @@ __device__ __forceinline__ bool softmax_block(const Ctx& c, const uint32_t (&sv)
   const float neg_m = st.m_ref == -INFINITY ? 0.f : -st.m_ref;
   uint32_t pk[32];
   float sum = 0.f;
-  if (nv == kBlock) {
 #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      const float e0 = ex2_approx(fmaf(__uint_as_float(sv[2 * t]), sl2, neg_m));
-      const float e1 = ex2_approx(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, neg_m));
-      sum += e0 + e1;
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
-      pk[t] = *reinterpret_cast<uint32_t*>(&b2);
-    }
-  } else {
-#pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      const float e0 = 2 * t < nv ? ex2_approx(fmaf(__uint_as_float(sv[2 * t]), sl2, neg_m)) : 0.f;
-      const float e1 = 2 * t + 1 < nv ? ex2_approx(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, neg_m)) : 0.f;
-      sum += e0 + e1;
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
-      pk[t] = *reinterpret_cast<uint32_t*>(&b2);
-    }
+  for (int t = 0; t < 32; ++t) {
+    float e0 = ex2_approx(fmaf(__uint_as_float(sv[2 * t]), sl2, neg_m));
+    float e1 = ex2_approx(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, neg_m));
+    e0 = 2 * t < nv ? e0 : 0.f;
+    e1 = 2 * t + 1 < nv ? e1 : 0.f;
+    sum += e0 + e1;
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+    pk[t] = *reinterpret_cast<uint32_t*>(&b2);
   }
   st.l += sum;
 
@@ -407,43 +392,36 @@ __device__ void score_softmax(const Ctx& c) {
     if (w.b < w.B && w.pre < w.e) prefetch_q_rows_l2(p, w.b, h);  // next segment's query
 
     SoftmaxState st{-INFINITY, 0.f};
-    for (int j = g.blk_lo; j < g.blk_hi; j += 2, ++pit) {
+    // one block per iteration (a single inlined copy of softmax_block); the
+    // two blocks of a pass share one S buffer, released after its last read
+    for (int j = g.blk_lo; j < g.blk_hi; ++j) {
+      const bool second = ((j - g.blk_lo) & 1) != 0;
+      const bool last_of_pass = second || j + 1 == g.blk_hi;
       const int sb = pit % kNS;
-      const bool has_b = j + 1 < g.blk_hi;
       int blk;
-      const int nv_a = block_rows(p, g, cur, j, c.lane, &blk);
-      const int nv_b = has_b ? block_rows(p, g, cur, j + 1, c.lane, &blk) : 0;
-      if (!warp_wait(bar_addr(c.bars->s_full[sb]), (pit / kNS) & 1u, c.wc)) {
-        alive = false;
-        break;
+      const int nv = block_rows(p, g, cur, j, c.lane, &blk);
+      if (!second) {
+        if (!warp_wait(bar_addr(c.bars->s_full[sb]), (pit / kNS) & 1u, c.wc)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
       }
-      tc_fence_after();
-      const uint32_t sa = c.tmem + lane_off + kSCol + sb * 128;
+      const uint32_t sa = c.tmem + lane_off + kSCol + sb * 128 + (second ? 64 : 0);
       uint32_t sv[64];
       tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_ld_wait();
-      if (!has_b) {
+      if (last_of_pass) {
         tc_fence_before();
         mbar_arrive(bar_addr(c.bars->s_empty[sb]));
+        ++pit;
       }
-      if (!softmax_block(c, sv, nv_a, j == g.blk_lo, sl2, pos, st, it, h, q4)) {
+      if (!softmax_block(c, sv, nv, j == g.blk_lo, sl2, pos, st, it, h, q4)) {
         alive = false;
         break;
       }
       ++it;
-      if (has_b) {
-        tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(bar_addr(c.bars->s_empty[sb]));
-        if (!softmax_block(c, sv, nv_b, false, sl2, pos, st, it, h, q4)) {
-          alive = false;
-          break;
-        }
-        ++it;
-      }
     }
     ++seg;
   }

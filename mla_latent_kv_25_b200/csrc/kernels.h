@@ -45,8 +45,12 @@ cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, 
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int B, int H, int S,
                            __nv_bfloat16* out, float* lse, cudaStream_t stream);
 
-cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* w_uk,
+// qmap: 3-D view {d 128, h H, b B} of q_nope with box {64, 1, 128}; wmap: 2-D
+// view {c 512, rows H*128} of W_UK with box {64, 64}; both 128 B swizzled.
+cudaError_t launch_absorb_q(const CUtensorMap& qmap, const CUtensorMap& wmap,
                             const __nv_bfloat16* q_rope, __nv_bfloat16* q_out, int ldq, int B,
-                            int H, cudaStream_t stream);
+                            int H, long long spin_limit, cudaStream_t stream);
+// Copies the absorption kernel's error word to *bits and clears it (synchronises `stream`).
+cudaError_t absorb_take_error(uint32_t* bits, cudaStream_t stream);
 
 }  // namespace mla

@@ -123,8 +123,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // phase completes (measured with a TMA streaming loop: 16 KB stages ran at
 // 36 GB/s per SM under try_wait and 64 GB/s under test_wait), which on the
 // decode pipeline's hand-offs costs more than the issue slots polling takes.
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const WaitCtx& w) {
-  if (mbar_test_wait(bar, parity)) return true;
+static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_test_wait(bar, parity)) return true;
@@ -137,6 +136,15 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const 
       }
     }
   }
+}
+
+// The first probe is inlined; the polling loop is one out-of-line copy shared
+// by every wait site, which keeps the kernel's hot code small (each role's
+// warps run different code, and instruction fetch misses showed up as the
+// main stall of the decode kernel).
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return wait_phase_slow(bar, parity, w);
 }
 
 // Whole-warp wait: every lane waits (each takes its own acquire); the warp

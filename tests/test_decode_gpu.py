@@ -143,17 +143,32 @@ def test_combine_matches_oracle():
     assert_close(to_np(lse).reshape(-1), rl, "combine lse", max_abs=1e-5)
 
 
-@pytest.mark.parametrize("B,H", [(1, 16), (5, 32), (64, 128)])
-def test_absorb_q_matches_oracle(B, H):
+@pytest.mark.parametrize("B,H,ldq", [(1, 16, 576), (5, 32, 576), (64, 128, 576), (130, 16, 640),
+                                     (257, 32, 576)])
+def test_absorb_q_matches_oracle(B, H, ldq):
+    """Tensor-core absorption: several 128-row tiles with a ragged last tile,
+    a padded row stride, every head count of the header's range ends."""
     w = inputs.make("v3", B=B, H=H, L=[1] * B, seed=33)
     qn, wu = w.q_nope.cuda(), w.w_uk.cuda()
     qr = w.q[:, :, 512:].contiguous().cuda()
-    q_out = torch.zeros((B, H, 576), dtype=torch.bfloat16, device="cuda")
+    q_out = torch.full((B, H, ldq), 7.0, dtype=torch.bfloat16, device="cuda")
     binding.mla_absorb_q(qn, wu, qr, q_out)
-    torch.cuda.synchronize()
+    assert binding.mla_absorb_get_error() == 0
     ref = oracle.absorb_q(w.q_nope, w.w_uk)
     assert_close(to_np(q_out[:, :, :512]).reshape(-1, 512), ref.reshape(-1, 512), "absorb")
-    assert torch.equal(q_out[:, :, 512:].cpu(), w.q[:, :, 512:])
+    assert torch.equal(q_out[:, :, 512:576].cpu(), w.q[:, :, 512:])
+    assert torch.all(q_out[:, :, 576:] == 7.0)  # padding past the row untouched
+
+
+def test_absorb_q_without_rope_leaves_tail():
+    B, H = 3, 16
+    w = inputs.make("v3", B=B, H=H, L=[1] * B, seed=34)
+    q_out = torch.full((B, H, 576), 5.0, dtype=torch.bfloat16, device="cuda")
+    binding.mla_absorb_q(w.q_nope.cuda(), w.w_uk.cuda(), None, q_out)
+    assert binding.mla_absorb_get_error() == 0
+    ref = oracle.absorb_q(w.q_nope, w.w_uk)
+    assert_close(to_np(q_out[:, :, :512]).reshape(-1, 512), ref.reshape(-1, 512), "absorb no-rope")
+    assert torch.all(q_out[:, :, 512:] == 5.0)
 
 
 # ---------------------------------------------------------------- full-size configs, sampled rows
