@@ -6,12 +6,12 @@
 //
 //   score CTA (rank 0)                           value CTA (rank 1)
 //   ------------------                           ------------------
-//   w0  TMA: cache rows of two 64-token blocks    w0  TMA: latent part of each block,
-//       per pass, one 64-column chunk at a time       half a block (4 chunks) at a time
-//       into a ring of [128 x 64] slots               into a ring of [64 x 256] slots
-//   w1  MMA: S = Q K^T for 128 tokens at once     w1  MMA: O += P V (A = P, B = V read
-//       (N = 128); latent part of Q in TMEM,          MN-major), N = 256 per instruction
-//       RoPE part of Q in shared memory           w2  zero V rows past seq_len
+//   w0  TMA: cache rows of three 64-token         w0  TMA: latent part of each block,
+//       blocks per pass, one 64-column chunk          half a block (4 chunks) at a time
+//       at a time into a ring of [192 x 64] slots     into a ring of [64 x 256] slots
+//   w1  MMA: S = Q K^T for 192 tokens at once     w1  MMA: O += P V (A = P, B = V read
+//       (N = 192); Q columns 0..255 in TMEM,          MN-major), N = 256 per instruction
+//       columns 256..575 in shared memory         w2  zero V rows past seq_len
 //   w4-7 softmax, thread h = head h: online       w4-7 thread h = head h: rescale O rows
 //       softmax in fp32 per 64-token block;           when the running max grew; final
 //       P (bf16) and the rescale factors are         O / l and lse, or an fp32 piece of
@@ -19,6 +19,11 @@
 //   w2-3 senders: staged records -> value CTA
 //       with st.async (overlapping the softmax)
 //
+// Why N = 192: inside this pipeline an MMA instruction costs roughly 100+
+// cycles to issue whatever its N, so 128-token passes ran the QK at half the
+// tensor pipe's rate; 192-token passes cut the instructions per block from 18
+// to 12.  Two 192-column S buffers leave TMEM room for only half of Q; the
+// rest of Q is an SS operand.
 // Heads are the M = 128 dimension of both contractions (padded with zero query
 // rows for H < 128).  The running max only moves when a block's max exceeds
 // it by more than 2^8 (log2 domain), so O is rarely rescaled.  Every wait is
@@ -43,27 +48,30 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 256;
-constexpr int kKChunks = 3;  // score CTA: 64-column chunks per K slot
-constexpr int kKSlots = 3;   // score CTA: ring of [128 tokens x 192 cols] slots (one pass = 3 slots)
+constexpr int kPassBlocks = 3;  // score CTA: blocks per QK pass, so N = 192 per MMA
+constexpr int kPassTok = kPassBlocks * 64;
+constexpr int kKSlots = 3;      // score CTA: ring of [192 tokens x 64 cols] slots, one column chunk each
 constexpr int kVSlots = 5;   // value CTA: ring of [64 tokens x 256 cols] half-block slots
 constexpr int kNP = 3;       // P records in flight
 constexpr int kNS = 2;       // S accumulators (128 columns each) in TMEM
 
 constexpr uint32_t kChunk = 64 * 128;          // one [64 rows x 64 bf16] swizzled chunk
-constexpr uint32_t kKPair = 2 * kChunk;         // one chunk of both blocks: [128 rows x 64 bf16]
-constexpr uint32_t kKSlot = kKChunks * kKPair;   // [128 rows x 192 bf16] as 3 swizzled [128 x 64] tiles
-static_assert(9 % kKChunks == 0, "a pass is a whole number of K slots");
+constexpr uint32_t kKSlot = kPassBlocks * kChunk;  // one column chunk of a pass: [192 rows x 64 bf16]
 constexpr uint32_t kVSlot = 4 * kChunk;         // [64 rows x 256 bf16]
 constexpr uint32_t kPBytes = 128 * 64 * 2;     // P [128 heads x 64 tokens] bf16
-constexpr uint32_t kQRopeBytes = 128 * 64 * 2; // RoPE part of Q [128 heads x 64] bf16
+constexpr uint32_t kQTile = 128 * 64 * 2;      // one 64-column chunk of Q [128 heads x 64] bf16
+constexpr int kQTmemChunks = 4;                 // Q columns 0..255 live in TMEM (TS operand)
+constexpr int kQSmemTiles = 9 - kQTmemChunks;   // columns 256..575 in shared memory (SS operand)
 constexpr uint32_t kMetaWarp = 400;            // per warp: alpha[32] m[32] l[32] flag + pad
 constexpr uint32_t kMetaBytes = 4 * kMetaWarp;
 constexpr float kRescaleThreshold = 8.0f;      // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 
-// TMEM columns of the score CTA: latent part of Q (512 bf16 = 256 columns), then S.
+// TMEM columns of the score CTA: Q columns 0..255 (bf16 pairs: 128 columns),
+// then two S buffers of kPassTok fp32 columns each.
 constexpr uint32_t kQCol = 0;
-constexpr uint32_t kSCol = 256;
+constexpr uint32_t kSCol = kQTmemChunks * 32;
+static_assert(kSCol + 2 * kPassTok <= 512, "TMEM columns");
 constexpr uint32_t kTmemCols = 512;
 
 struct Barriers {
@@ -82,8 +90,8 @@ static_assert(sizeof(Barriers) <= 1024, "barrier block too large");
 
 // shared-memory offsets from the 1024-aligned base
 constexpr uint32_t kRegion = 1024;
-__host__ __device__ constexpr uint32_t q_rope_off() { return kRegion; }
-__host__ __device__ constexpr uint32_t k_slot_off(int s) { return kRegion + kQRopeBytes + s * kKSlot; }
+__host__ __device__ constexpr uint32_t q_tile_off(int t) { return kRegion + t * kQTile; }
+__host__ __device__ constexpr uint32_t k_slot_off(int s) { return kRegion + kQSmemTiles * kQTile + s * kKSlot; }
 // score CTA staging of the P records and factors before the bulk copy
 __host__ __device__ constexpr uint32_t p_stage_off(int r) { return k_slot_off(kKSlots) + r * kPBytes; }
 __host__ __device__ constexpr uint32_t meta_stage_off(int r) {
@@ -101,7 +109,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(k_slot_off(0) % 1024 == 0 && p_rec_off(0) % 1024 == 0 && p_stage_off(0) % 1024 == 0,
               "swizzle atoms need 1024 B");
 
-constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false, false);  // S[128x128] = Q . K^T
+constexpr uint32_t kIdescQK = idesc_bf16(128, kPassTok, false, false);  // S[128 x 192] = Q . K^T
 constexpr uint32_t kIdescPV = idesc_bf16(128, 256, false, true);   // O[128x256] += P . V
 
 struct Ctx {
@@ -155,9 +163,9 @@ __device__ __forceinline__ int block_rows(const DecodeParams& p, const Segment& 
 
 // ============================================================ score CTA roles
 
-// Two consecutive blocks of a segment form one pass (the second may be
-// absent at the end of the segment); each pass streams its 9 column chunks
-// through the slot ring.
+// kPassBlocks consecutive blocks of a segment form one pass (fewer at the end
+// of the segment); each pass streams its 9 column chunks through the slot
+// ring, one chunk of all the pass's blocks per slot.
 __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   const DecodeParams& p = *c.p;
   SegWalker w;
@@ -169,20 +177,19 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   if (c.lane == 0) prefetch_tmap(tmap);
   while (alive && w.next(g)) {
     cur.reset(p, g);
-    for (int j = g.blk_lo; alive && j < g.blk_hi; j += 2) {
-      int blk_a, blk_b = 0;
-      const int nv_a = block_rows(p, g, cur, j, c.lane, &blk_a);
-      const bool has_b = j + 1 < g.blk_hi;
-      int nv_b = 0;
-      if (has_b) nv_b = block_rows(p, g, cur, j + 1, c.lane, &blk_b);
-      if (c.lane == 0) {
-        if (nv_a == 0 && g.len > j * kBlock) atomicOr(p.err, kErrBadBlock);
-        if (has_b && nv_b == 0) atomicOr(p.err, kErrBadBlock);
+    for (int j = g.blk_lo; alive && j < g.blk_hi; j += kPassBlocks) {
+      const int nb = min(kPassBlocks, g.blk_hi - j);
+      int blk[kPassBlocks];
+#pragma unroll
+      for (int k = 0; k < kPassBlocks; ++k) {
+        blk[k] = 0;
+        if (k < nb) {
+          // every block of the segment holds at least one token: 0 rows = bad id
+          if (block_rows(p, g, cur, j + k, c.lane, &blk[k]) == 0 && c.lane == 0)
+            atomicOr(p.err, kErrBadBlock);
+        }
       }
-      // one K slot = kKChunks column chunks of both blocks: few, large TMA
-      // transactions per barrier (per-SM TMA throughput grows with the bytes
-      // one barrier tracks)
-      for (int i = 0; i < 9 / kKChunks; ++i, ++cit) {
+      for (int ch = 0; ch < 9; ++ch, ++cit) {
         const int s = cit % kKSlots;
         if (!warp_wait(bar_addr(c.bars->k_empty[s]), ((cit / kKSlots) & 1u) ^ 1u, c.wc)) {
           alive = false;
@@ -190,14 +197,11 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
         }
         if (c.lane == 0) {
           const uint32_t full = bar_addr(c.bars->k_full[s]);
-          mbar_arrive_expect_tx(full, (has_b ? 2u : 1u) * kKChunks * kChunk);
+          mbar_arrive_expect_tx(full, static_cast<uint32_t>(nb) * kChunk);
           const uint32_t dst = c.base + k_slot_off(s);
 #pragma unroll
-          for (int q = 0; q < kKChunks; ++q) {
-            const int ch = i * kKChunks + q;
-            tma_load_2d(dst + q * kKPair, tmap, ch * 64, blk_a * kBlock, full);
-            if (has_b) tma_load_2d(dst + q * kKPair + kChunk, tmap, ch * 64, blk_b * kBlock, full);
-          }
+          for (int k = 0; k < kPassBlocks; ++k)
+            if (k < nb) tma_load_2d(dst + k * kChunk, tmap, ch * 64, blk[k] * kBlock, full);
         }
         __syncwarp();
       }
@@ -214,88 +218,93 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   }
 }
 
+// The whole warp walks the segments (the walker uses warp collectives), but
+// each segment's issue loop runs in one single-thread region of lane 0:
+// issuing a slot's MMAs from a lane-0 branch that the warp enters and leaves
+// every slot measured about twice the cycles per MMA of a single-thread loop.
+__device__ bool score_mma_segment(const Ctx& c, const Segment& g, uint32_t seg, uint32_t& cit,
+                                  uint32_t& pit) {
+  const uint32_t tmem = c.tmem;
+  const uint32_t qs = c.base + q_tile_off(0);
+  const uint32_t kbase = c.base + k_slot_off(0);
+  Barriers* bars = c.bars;
+  if (!wait_phase(bar_addr(bars->q_ready), seg & 1u, c.wc)) return false;
+  tc_fence_after();
+  for (int j = g.blk_lo; j < g.blk_hi; j += kPassBlocks, ++pit) {
+    const int sb = pit % kNS;
+    if (!wait_phase(bar_addr(bars->s_empty[sb]), ((pit / kNS) & 1u) ^ 1u, c.wc)) return false;
+    const uint32_t d = tmem + kSCol + sb * kPassTok;
+    for (int ch = 0; ch < 9; ++ch, ++cit) {
+      const int s = cit % kKSlots;
+      if (!wait_phase(bar_addr(bars->k_full[s]), (cit / kKSlots) & 1u, c.wc)) return false;
+      tc_fence_after();
+      const uint32_t tile = kbase + s * kKSlot;
+      if (ch < kQTmemChunks) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(d, tmem + kQCol + 32 * ch + 8 * kk, sw128_desc(tile + kk * 32, 16, 1024), kIdescQK,
+                 (ch | kk) ? 1u : 0u);
+      } else {
+        const uint32_t qt = qs + (ch - kQTmemChunks) * kQTile;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(d, sw128_desc(qt + kk * 32, 16, 1024), sw128_desc(tile + kk * 32, 16, 1024), kIdescQK, 1u);
+      }
+      mma_commit(bar_addr(bars->k_empty[s]));
+    }
+    mma_commit(bar_addr(bars->s_full[sb]));
+  }
+  mma_commit(bar_addr(bars->q_free));
+  return true;
+}
+
 __device__ void score_mma(const Ctx& c) {
   const DecodeParams& p = *c.p;
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
   uint32_t cit = 0, pit = 0, seg = 0;
-  const uint32_t qrope = c.base + q_rope_off();
   while (w.next(g)) {
-    if (!warp_wait(bar_addr(c.bars->q_ready), seg & 1u, c.wc)) return;
-    tc_fence_after();
-    for (int j = g.blk_lo; j < g.blk_hi; j += 2, ++pit) {
-      const int sb = pit % kNS;
-      if (!warp_wait(bar_addr(c.bars->s_empty[sb]), ((pit / kNS) & 1u) ^ 1u, c.wc)) return;
-      const uint32_t d = c.tmem + kSCol + sb * 128;
-      for (int i = 0; i < 9 / kKChunks; ++i, ++cit) {
-        const int s = cit % kKSlots;
-        if (!warp_wait(bar_addr(c.bars->k_full[s]), (cit / kKSlots) & 1u, c.wc)) return;
-        tc_fence_after();
-        if (c.lane == 0) {
-#pragma unroll
-          for (int q = 0; q < kKChunks; ++q) {
-            const int ch = i * kKChunks + q;
-            const uint32_t tile = c.base + k_slot_off(s) + q * kKPair;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t b = sw128_desc(tile + kk * 32, 16, 1024);
-              if (ch < 8)
-                mma_ts(d, c.tmem + kQCol + 32 * ch + 8 * kk, b, kIdescQK, (ch | kk) ? 1u : 0u);
-              else
-                mma_ss(d, sw128_desc(qrope + kk * 32, 16, 1024), b, kIdescQK, 1u);
-            }
-          }
-          mma_commit(bar_addr(c.bars->k_empty[s]));
-        }
-        __syncwarp();
-      }
-      if (c.lane == 0) mma_commit(bar_addr(c.bars->s_full[sb]));
-      __syncwarp();
-    }
-    if (c.lane == 0) mma_commit(bar_addr(c.bars->q_free));
-    __syncwarp();
+    int ok = 1;
+    if (c.lane == 0) ok = score_mma_segment(c, g, seg, cit, pit) ? 1 : 0;
+    if (!__shfl_sync(0xffffffffu, ok, 0)) return;
     ++seg;
   }
 }
 
-// Query row of sequence b for head h: the latent part (512 bf16) into TMEM
-// lane h as 256 packed columns, the RoPE part (64 bf16) into the swizzled
-// [128 x 64] K-major tile in shared memory.  Loads run four chunks ahead.
+// Query row of sequence b for head h: columns 0..255 into TMEM lane h as 128
+// packed columns (the TS operand of the first four column chunks), columns
+// 256..575 into five swizzled [128 x 64] K-major tiles in shared memory (the
+// SS operand of the last five).
 __device__ __forceinline__ void load_q_rows(const DecodeParams& p, int b, int h, uint32_t taddr,
-                                            uint8_t* qrope) {
+                                            uint8_t* qtiles) {
   const bool live = h < p.H;
   const uint4* src = reinterpret_cast<const uint4*>(p.q + (size_t(b) * p.H + (live ? h : 0)) * kRow);
   const uint4 z = make_uint4(0, 0, 0, 0);
-  uint4 rope[8];
+  const uint32_t swz = static_cast<uint32_t>(h & 7);
 #pragma unroll
-  for (int v = 0; v < 8; ++v) rope[v] = live ? __ldg(src + 64 + v) : z;
-  uint4 buf[4][8];
+  for (int ch = 0; ch < 9; ++ch) {
+    uint4 v8[8];
 #pragma unroll
-  for (int ch = 0; ch < 4; ++ch)
+    for (int v = 0; v < 8; ++v) v8[v] = live ? __ldg(src + ch * 8 + v) : z;
+    if (ch < kQTmemChunks) {
+      uint32_t r[32];
 #pragma unroll
-    for (int v = 0; v < 8; ++v) buf[ch][v] = live ? __ldg(src + ch * 8 + v) : z;
+      for (int v = 0; v < 8; ++v) {
+        r[4 * v] = v8[v].x;
+        r[4 * v + 1] = v8[v].y;
+        r[4 * v + 2] = v8[v].z;
+        r[4 * v + 3] = v8[v].w;
+      }
+      tmem_st32(taddr + 32 * ch, r);
+    } else {
+      uint8_t* row = qtiles + (ch - kQTmemChunks) * kQTile + h * 128;
 #pragma unroll
-  for (int ch = 0; ch < 8; ++ch) {
-    uint32_t r[32];
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      r[4 * v] = buf[ch % 4][v].x;
-      r[4 * v + 1] = buf[ch % 4][v].y;
-      r[4 * v + 2] = buf[ch % 4][v].z;
-      r[4 * v + 3] = buf[ch % 4][v].w;
-    }
-    tmem_st32(taddr + 32 * ch, r);
-    if (ch + 4 < 8) {
-#pragma unroll
-      for (int v = 0; v < 8; ++v) buf[ch % 4][v] = live ? __ldg(src + (ch + 4) * 8 + v) : z;
+      for (int v = 0; v < 8; ++v)
+        *reinterpret_cast<uint4*>(row + ((static_cast<uint32_t>(v) ^ swz) << 4)) = v8[v];
     }
   }
-#pragma unroll
-  for (int v = 0; v < 8; ++v)
-    *reinterpret_cast<uint4*>(qrope + h * 128 + ((v ^ (h & 7)) << 4)) = rope[v];
 }
-
 __device__ __forceinline__ void prefetch_q_rows_l2(const DecodeParams& p, int b, int h) {
   if (h >= p.H) return;
   const char* src = reinterpret_cast<const char*>(p.q + (size_t(b) * p.H + h) * kRow);
@@ -371,7 +380,7 @@ __device__ void score_softmax(const Ctx& c) {
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
   const float sl2 = p.softmax_scale * kLog2e;
   const bool pos = sl2 >= 0.f;
-  uint8_t* qrope = c.gbase + q_rope_off();
+  uint8_t* qtiles = c.gbase + q_tile_off(0);
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
@@ -384,7 +393,7 @@ __device__ void score_softmax(const Ctx& c) {
       if (!warp_wait(bar_addr(c.bars->q_free), (seg - 1) & 1u, c.wc)) break;
       tc_fence_after();
     }
-    load_q_rows(p, g.b, h, c.tmem + lane_off + kQCol, qrope);
+    load_q_rows(p, g.b, h, c.tmem + lane_off + kQCol, qtiles);
     fence_proxy_async_smem();
     tmem_st_wait();
     tc_fence_before();
@@ -393,21 +402,21 @@ __device__ void score_softmax(const Ctx& c) {
 
     SoftmaxState st{-INFINITY, 0.f};
     // one block per iteration (a single inlined copy of softmax_block); the
-    // two blocks of a pass share one S buffer, released after its last read
+    // blocks of a pass share one S buffer, released after its last read
     for (int j = g.blk_lo; j < g.blk_hi; ++j) {
-      const bool second = ((j - g.blk_lo) & 1) != 0;
-      const bool last_of_pass = second || j + 1 == g.blk_hi;
+      const int k = (j - g.blk_lo) % kPassBlocks;
+      const bool last_of_pass = k == kPassBlocks - 1 || j + 1 == g.blk_hi;
       const int sb = pit % kNS;
       int blk;
       const int nv = block_rows(p, g, cur, j, c.lane, &blk);
-      if (!second) {
+      if (k == 0) {
         if (!warp_wait(bar_addr(c.bars->s_full[sb]), (pit / kNS) & 1u, c.wc)) {
           alive = false;
           break;
         }
         tc_fence_after();
       }
-      const uint32_t sa = c.tmem + lane_off + kSCol + sb * 128 + (second ? 64 : 0);
+      const uint32_t sa = c.tmem + lane_off + kSCol + sb * kPassTok + 64 * k;
       uint32_t sv[64];
       tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
@@ -561,6 +570,49 @@ __device__ void value_fixup(const Ctx& c) {
   }
 }
 
+// As for the score MMA warp: each segment's issue loop is one single-thread
+// region of lane 0.
+__device__ bool value_mma_segment(const Ctx& c, const Segment& g, uint32_t seg, uint32_t& it,
+                                  uint32_t& vit, uint32_t& ncorr) {
+  if (seg > 0) {
+    if (!wait_phase(bar_addr(c.bars->o_free), (seg - 1) & 1u, c.wc)) return false;
+    tc_fence_after();
+  }
+  for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
+    const int r = it % kNP;
+    if (!wait_phase(bar_addr(c.bars->p_full[r]), (it / kNP) & 1u, c.wc)) return false;
+    const bool first = (j == g.blk_lo);
+    const uint8_t* meta = c.gbase + meta_rec_off(r);
+    uint32_t any = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) any |= reinterpret_cast<const uint32_t*>(meta + q * kMetaWarp)[96];
+    if (any && !first) {
+      // hand O over for rescaling once every MMA issued so far (the previous
+      // block's PV) has completed, and take it back when rescaled
+      mma_commit(bar_addr(c.bars->pv_prev));
+      if (!wait_phase(bar_addr(c.bars->corr_done), ncorr & 1u, c.wc)) return false;
+      ++ncorr;
+    }
+    fence_proxy_async_smem();
+    const uint32_t pa = c.base + p_rec_off(r);
+    for (int n = 0; n < 2; ++n, ++vit) {
+      const int s = vit % kVSlots;
+      if (!wait_phase(bar_addr(c.bars->v_full[s]), (vit / kVSlots) & 1u, c.wc)) return false;
+      if (!wait_phase(bar_addr(c.bars->v_fixed[s]), (vit / kVSlots) & 1u, c.wc)) return false;
+      tc_fence_after();
+      const uint32_t va = c.base + v_slot_off(s);
+#pragma unroll
+      for (int k = 0; k < kBlock / 16; ++k)
+        mma_ss(c.tmem + 256 * n, sw128_desc(pa + k * 32, 16, 1024),
+               sw128_desc(va + k * 2048, kChunk, 1024), kIdescPV, (k > 0 || !first) ? 1u : 0u);
+      mma_commit(bar_addr(c.bars->v_empty[s]));
+    }
+    mma_commit_mc(bar_addr(c.bars->p_empty[r]), 0x1);
+    if (j == g.blk_hi - 1) mma_commit(bar_addr(c.bars->o_ready));  // O final for this segment
+  }
+  return true;
+}
+
 __device__ void value_mma(const Ctx& c) {
   const DecodeParams& p = *c.p;
   SegWalker w;
@@ -568,49 +620,9 @@ __device__ void value_mma(const Ctx& c) {
   Segment g;
   uint32_t it = 0, vit = 0, seg = 0, ncorr = 0;
   while (w.next(g)) {
-    if (seg > 0) {
-      if (!warp_wait(bar_addr(c.bars->o_free), (seg - 1) & 1u, c.wc)) return;
-      tc_fence_after();
-    }
-    for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
-      const int r = it % kNP;
-      if (!warp_wait(bar_addr(c.bars->p_full[r]), (it / kNP) & 1u, c.wc)) return;
-      const bool first = (j == g.blk_lo);
-      const uint8_t* meta = c.gbase + meta_rec_off(r);
-      uint32_t any = 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) any |= reinterpret_cast<const uint32_t*>(meta + q * kMetaWarp)[96];
-      if (any && !first) {
-        // hand O over for rescaling once every MMA issued so far (the previous
-        // block's PV) has completed, and take it back when rescaled
-        if (c.lane == 0) mma_commit(bar_addr(c.bars->pv_prev));
-        __syncwarp();
-        if (!warp_wait(bar_addr(c.bars->corr_done), ncorr & 1u, c.wc)) return;
-        ++ncorr;
-      }
-      fence_proxy_async_smem();
-      const uint32_t pa = c.base + p_rec_off(r);
-      for (int n = 0; n < 2; ++n, ++vit) {
-        const int s = vit % kVSlots;
-        if (!warp_wait(bar_addr(c.bars->v_full[s]), (vit / kVSlots) & 1u, c.wc)) return;
-        if (!warp_wait(bar_addr(c.bars->v_fixed[s]), (vit / kVSlots) & 1u, c.wc)) return;
-        tc_fence_after();
-        if (c.lane == 0) {
-          const uint32_t va = c.base + v_slot_off(s);
-#pragma unroll
-          for (int k = 0; k < kBlock / 16; ++k)
-            mma_ss(c.tmem + 256 * n, sw128_desc(pa + k * 32, 16, 1024),
-                   sw128_desc(va + k * 2048, kChunk, 1024), kIdescPV, (k > 0 || !first) ? 1u : 0u);
-          mma_commit(bar_addr(c.bars->v_empty[s]));
-        }
-        __syncwarp();
-      }
-      if (c.lane == 0) {
-        mma_commit_mc(bar_addr(c.bars->p_empty[r]), 0x1);
-        if (j == g.blk_hi - 1) mma_commit(bar_addr(c.bars->o_ready));  // O final for this segment
-      }
-      __syncwarp();
-    }
+    int ok = 1;
+    if (c.lane == 0) ok = value_mma_segment(c, g, seg, it, vit, ncorr) ? 1 : 0;
+    if (!__shfl_sync(0xffffffffu, ok, 0)) return;
     ++seg;
   }
 }

@@ -123,15 +123,19 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // phase completes (measured with a TMA streaming loop: 16 KB stages ran at
 // 36 GB/s per SM under try_wait and 64 GB/s under test_wait), which on the
 // decode pipeline's hand-offs costs more than the issue slots polling takes.
-static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+// Arguments by value: a reference would force the caller's context into
+// local memory, and every asm statement with a "memory" clobber (all the
+// barrier, TMA and MMA wrappers here) would then reload it.
+static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, long long limit,
+                                                    uint32_t* err, volatile int* abort) {
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_test_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
-      if (*w.abort) return false;
-      if (clock64() - t0 > w.limit) {
-        atomicOr(w.err, kErrTimeout);
-        *w.abort = 1;
+      if (*abort) return false;
+      if (clock64() - t0 > limit) {
+        atomicOr(err, kErrTimeout);
+        *abort = 1;
         return false;
       }
     }
@@ -140,11 +144,10 @@ static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parit
 
 // The first probe is inlined; the polling loop is one out-of-line copy shared
 // by every wait site, which keeps the kernel's hot code small (each role's
-// warps run different code, and instruction fetch misses showed up as the
-// main stall of the decode kernel).
+// warps run different code).
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_test_wait(bar, parity)) return true;
-  return wait_phase_slow(bar, parity, w);
+  return wait_phase_slow(bar, parity, w.limit, w.err, w.abort);
 }
 
 // Whole-warp wait: every lane waits (each takes its own acquire); the warp
