@@ -65,6 +65,28 @@ def dist_env():
     return world, rank, local
 
 
+def rank_seed(workload: str, rank: int) -> int:
+    """Each replica decodes its own batch: the workload's seed offset by rank."""
+    return inputs.CONFIGS[workload]["seed"] + 1000 * rank
+
+
+def max_over_ranks(values, device):
+    """Elementwise max over all ranks of the process group (a no-op for one
+    process); every rank gets the result.  Timings are reported as the slowest
+    rank's."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_rate(bytes_per_rank_step: float, world: int, step_ms: float) -> float:
+    """Whole-job GB/s: the bytes every rank processed per step over the
+    (max-over-ranks) step time."""
+    return bytes_per_rank_step * world / (step_ms * 1e-3) / 1e9
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -190,7 +212,7 @@ def run_ours(args, world, rank, local):
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
-    w = inputs.make(args.workload, seed=inputs.CONFIGS[args.workload]["seed"] + 1000 * rank)
+    w = inputs.make(args.workload, seed=rank_seed(args.workload, rank))
     d = binding.to_device(w, dev)
     B, H = w.B, w.H
     stream = torch.cuda.current_stream(dev)
@@ -262,10 +284,7 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("device error during timing")
 
     step_ms = ms / K
-    if world > 1:
-        t = torch.tensor([step_ms, dec_ms, e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms, dec_ms, e2e_ms = (float(x) for x in t.tolist())
+    step_ms, dec_ms, e2e_ms = max_over_ranks([step_ms, dec_ms, e2e_ms], dev)
 
     res = None
     if rank == 0:
@@ -273,7 +292,7 @@ def run_ours(args, world, rank, local):
         hbm = float(peaks["hbm_gbs"])
         tens = float(peaks["bf16_tflops"])
         step_bytes = dec_b + abs_b
-        value = step_bytes * world / (step_ms * 1e-3) / 1e9
+        value = job_rate(step_bytes, world, step_ms)
         achieved = dec_b / (dec_ms * 1e-3) / 1e9
         dec_tflops = dec_f / (dec_ms * 1e-3) / 1e12
         t_hbm = dec_b / (hbm * 1e9)
@@ -314,7 +333,7 @@ def run_ours(args, world, rank, local):
             "tflops": round((dec_f + abs_f) * world / (step_ms * 1e-3) / 1e12, 2),
             "decode_tflops": round(dec_tflops, 2),
             "roofline": roof,
-            "e2e": {"value": round(step_bytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "e2e": {"value": round(job_rate(step_bytes, world, e2e_ms), 1), "unit": "GB/s",
                     "ms_per_step": round(e2e_ms, 5),
                     "h2d_bytes_per_step": int(h_qn.numel() * 2 + h_qr.numel() * 2),
                     "d2h_bytes_per_step": int(h_out.numel() * 2 + h_lse.numel() * 4)},
