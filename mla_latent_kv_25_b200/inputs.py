@@ -52,6 +52,8 @@ class Workload:
     # inputs of the query absorption step (q_abs = q_nope . W_UK[h])
     q_nope: Optional[torch.Tensor] = None   # bf16 [B,H,128]
     w_uk: Optional[torch.Tensor] = None     # bf16 [H,128,512]
+    # input of the output absorption step (out_h = W_UV[h] . o_latent)
+    w_uv: Optional[torch.Tensor] = None     # bf16 [H,128,512]
     extras: dict = field(default_factory=dict)
 
     @property
@@ -227,7 +229,7 @@ def make(name: str, *, seed: Optional[int] = None, B: Optional[int] = None,
                 cache_t[blk, r0:, :] = 0x7F  # an E4M3 NaN code
                 k_rope_t[blk, r0:, :] = float(tail_fill)
 
-    q_nope = w_uk = None
+    q_nope = w_uk = w_uv = None
     if with_absorb:
         # q_abs = q_nope . W_UK[h]; spreads chosen so q_abs has the same spread
         # as the directly drawn q_abs above.
@@ -237,11 +239,13 @@ def make(name: str, *, seed: Optional[int] = None, B: Optional[int] = None,
             qn_std, w_std = 1.0, 1.0 / math.sqrt(D_NOPE)
         q_nope = _randn(g, (Bn, Hn, D_NOPE), qn_std).to(torch.bfloat16)
         w_uk = _randn(g, (Hn, D_NOPE, D_C), w_std).to(torch.bfloat16)
+        # drawn last, so every earlier draw is unchanged by its presence
+        w_uv = _randn(g, (Hn, D_NOPE, D_C), 1.0 / math.sqrt(D_C)).to(torch.bfloat16)
 
     return Workload(name=name, B=Bn, H=Hn, seq_lens=seq_lens, block_table=table,
                     num_blocks=NB, cache_dtype=kind, cache=cache_t, k_rope=k_rope_t,
                     block_scale=scale_t, q=q, softmax_scale=1.0 / math.sqrt(D_NOPE + D_R),
-                    seed=int(spec["seed"]), q_nope=q_nope, w_uk=w_uk, extras=extras)
+                    seed=int(spec["seed"]), q_nope=q_nope, w_uk=w_uk, w_uv=w_uv, extras=extras)
 
 
 def relocate(w: Workload, seed: int) -> Workload:

@@ -7,7 +7,7 @@ with, or called by, the CUDA path.
 Parts:
   * ``mla_oracle.c`` (compiled to ``_build/liboracle.so``): the plain
     definition of absorbed decode attention over the paged latent cache, the
-    log-sum-exp merge of split pieces, the query absorption, and the bf16 /
+    log-sum-exp merge of split pieces, the query and output absorptions, and the bf16 /
     OCP E4M3 decoders.
   * ``naive.py``: the unabsorbed form (per-head keys and values formed from
     the latent with W_UK / W_UV, RoPE on the decoupled part only, plain
@@ -62,6 +62,8 @@ def lib():
             L.orc_combine.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, vp, vp]
             L.orc_absorb_q.restype = None
             L.orc_absorb_q.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, vp]
+            L.orc_absorb_o.restype = None
+            L.orc_absorb_o.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, vp]
             L.orc_bf16_to_f64.restype = ctypes.c_double
             L.orc_bf16_to_f64.argtypes = [ctypes.c_uint16]
             L.orc_e4m3_to_f64.restype = ctypes.c_double
@@ -175,6 +177,16 @@ def combine(o_part, lse_part):
     lse = np.zeros((R,), dtype=np.float64)
     lib().orc_combine(_ptr(op), _ptr(lp), R, S, _ptr(out), _ptr(lse))
     return out, lse
+
+
+def absorb_o(o_latent, w_uv):
+    """out[b,h,d] = sum_c W_UV[h,d,c] * o_latent[b,h,c] in double; bf16 inputs."""
+    ol = _np(o_latent, np.uint16)
+    wv = _np(w_uv, np.uint16)
+    B, H = int(ol.shape[0]), int(ol.shape[1])
+    out = np.zeros((B, H, 128), dtype=np.float64)
+    lib().orc_absorb_o(_ptr(ol), _ptr(wv), B, H, _ptr(out))
+    return out
 
 
 def absorb_q(q_nope, w_uk):

@@ -247,6 +247,26 @@ void orc_absorb_q(const uint16_t *q_nope, const uint16_t *w_uk, int B, int H, do
         }
 }
 
+/*
+ * Output absorption ("Empirical Gains": W^UV is absorbed into the output
+ * projection, so the head's value vector is never formed per token):
+ *     out[b,h,d] = sum_{c<512} W_UV[h,d,c] * o_latent[b,h,c],   d < 128
+ * o_latent: bf16 [B,H,512]; w_uv: bf16 [H,128,512]; out: double [B,H,128].
+ */
+void orc_absorb_o(const uint16_t *o_lat, const uint16_t *w_uv, int B, int H, double *out) {
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const uint16_t *o = o_lat + ((int64_t)b * H + h) * ORC_DC;
+            double *dst = out + ((int64_t)b * H + h) * 128;
+            for (int d = 0; d < 128; ++d) {
+                const uint16_t *w = w_uv + ((int64_t)h * 128 + d) * ORC_DC;
+                double acc = 0.0;
+                for (int c = 0; c < ORC_DC; ++c) acc += orc_bf16_to_f64(w[c]) * orc_bf16_to_f64(o[c]);
+                dst[d] = acc;
+            }
+        }
+}
+
 int orc_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

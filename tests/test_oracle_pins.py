@@ -303,6 +303,59 @@ def test_absorb_q_matches_library_matmul():
     assert np.max(np.abs(got - ref)) < 1e-12
 
 
+def test_absorb_o_matches_library_matmul():
+    """Output absorption (Empirical Gains: W^UV folded into the output
+    projection): out[b,h,:] = W_UV[h] . o_latent[b,h,:]."""
+    w = inputs.make("v3", B=3, H=8, L=[1, 1, 1], seed=18)
+    o = (torch.randn((3, 8, 512), generator=torch.Generator().manual_seed(3)) * 0.05).to(torch.bfloat16)
+    ref = torch.einsum("hdc,bhc->bhd", w.w_uv.double(), o.double()).numpy()
+    got = oracle.absorb_o(o, w.w_uv)
+    assert got.shape == (3, 8, 128)
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_absorb_o_one_hot_rows_select_latent_columns():
+    """W_UV[h][d] = e_{4d + h % 4} picks one latent column per output: exact."""
+    B, H = 2, 4
+    w_uv = torch.zeros((H, 128, 512), dtype=torch.bfloat16)
+    for h in range(H):
+        for d in range(128):
+            w_uv[h, d, 4 * d + h % 4] = 1.0
+    o = torch.randn((B, H, 512), generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    got = oracle.absorb_o(o, w_uv)
+    for h in range(H):
+        assert np.array_equal(got[:, h, :], o[:, h, (h % 4)::4].double().numpy())
+
+
+def test_absorbed_decode_then_output_absorption_equals_naive_heads():
+    """Chaining the two absorbed steps on bf16-rounded inputs reproduces the
+    naive per-head attention output (the unabsorbed form) to bf16 input
+    rounding: the decode in f64 on the cache, then W_UV on its output."""
+    H, L = 16, 200
+    raw = inputs.raw_tiny_fp32(seed=1, H=H, L=L)
+    raw = {k: v.double().numpy() for k, v in raw.items()}
+    scale = 1.0 / math.sqrt(192)
+    o_naive, _ = naive.naive_mha(raw["c_kv"], raw["k_r"], raw["q_nope"], raw["q_r"],
+                                 raw["w_uk"], raw["w_uv"], scale, q_pos=L - 1)
+    k_rot = naive.rope(raw["k_r"], np.arange(L))
+    rows = np.concatenate([raw["c_kv"], k_rot], axis=1)
+    cache, table, NB = _paged_f64(rows, seed=7)
+    q_abs = np.einsum("hd,hdc->hc", raw["q_nope"], raw["w_uk"])
+    q = np.concatenate([q_abs, naive.rope(raw["q_r"], np.full(H, L - 1))], axis=1)[None]
+    o_lat, _ = oracle.decode_units(q=q, q_kind="f64", cache=cache, cache_kind="f64",
+                                   block_table=table, seq_lens=np.array([L], np.int32),
+                                   num_blocks=NB, softmax_scale=scale, units=oracle.all_units(1, H))
+    o_bf = torch.from_numpy(o_lat.reshape(1, H, 512)).to(torch.bfloat16)
+    w_uv_bf = torch.from_numpy(raw["w_uv"]).to(torch.bfloat16)
+    got = oracle.absorb_o(o_bf, w_uv_bf)[0]
+    # bf16 rounding of o_latent and W_UV only: relative error a few 2^-9
+    err = np.linalg.norm(got - o_naive) / np.linalg.norm(o_naive)
+    assert err < 1e-2
+    # and without the rounding the chain is exact
+    exact = np.einsum("hdc,hc->hd", raw["w_uv"], o_lat.reshape(H, 512))
+    assert np.max(np.abs(exact - o_naive)) < 1e-10
+
+
 # ---------------------------------------------------------------- page numbers
 
 def test_cache_size_closed_forms_match_page_values():
