@@ -76,7 +76,19 @@ mla_status_t mla_absorb_q(const void *q_nope, const void *w_uk, const void *q_ro
                           void *q_out, int ldq, int B, int H, void *stream);
 
 /*
- * mla_absorb_get_error - device error bits of the mla_absorb_q launches since
+ * mla_absorb_o - the output side of the absorption ("Empirical Gains": W^UV is
+ * absorbed into the output projection, so per-head values are never formed):
+ *     out[(b*H + h)*ldo + d] = sum_{c<512} w_uv[h,d,c] * o_latent[b,h,c],  d < 128
+ * o_latent: bf16 [B,H,512] (e.g. mla_decode's out); w_uv: bf16 [H,128,512];
+ * out: bf16 rows of stride ldo elements (ldo >= 128, a multiple of 8).
+ * fp32 accumulation (tensor cores), one bf16 rounding.  B >= 1; H in
+ * {16,32,...,128}.  All pointers 16-byte aligned; o_latent and w_uv dense.
+ */
+mla_status_t mla_absorb_o(const void *o_latent, const void *w_uv, void *out, int ldo, int B,
+                          int H, void *stream);
+
+/*
+ * mla_absorb_get_error - device error bits of the mla_absorb_q / mla_absorb_o launches since
  * the last call (MLA_DEVERR_TIMEOUT when a bounded wait in the kernel gave up;
  * the affected rows are then not written).  Synchronises `stream` and clears
  * the bits.  MLA_ERR_INVALID_ARG if err_bits is NULL.

@@ -29,7 +29,7 @@ DEVERR_SEQ_TOO_LONG = 0x2
 DEVERR_TIMEOUT = 0x4
 
 # every symbol include/mla.h declares
-EXPORTS = ("mla_absorb_q", "mla_absorb_get_error", "mla_decode_workspace_bytes", "mla_decode",
+EXPORTS = ("mla_absorb_q", "mla_absorb_o", "mla_absorb_get_error", "mla_decode_workspace_bytes", "mla_decode",
            "mla_combine", "mla_get_device_error", "mla_status_string", "mla_num_sms",
            "mla_decode_noalloc")
 
@@ -57,6 +57,8 @@ def load():
         vp, i32, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         L.mla_absorb_q.restype = i32
         L.mla_absorb_q.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
+        L.mla_absorb_o.restype = i32
+        L.mla_absorb_o.argtypes = [vp, vp, vp, i32, i32, i32, vp]
         L.mla_absorb_get_error.restype = i32
         L.mla_absorb_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_decode_workspace_bytes.restype = u64
@@ -141,6 +143,19 @@ def mla_absorb_q(q_nope, w_uk, q_rope, q_out, stream=None):
     _check("mla_absorb_q", load().mla_absorb_q(_ptr(q_nope), _ptr(w_uk), _ptr(q_rope), _ptr(q_out),
                                                ldq, B, H, _stream(stream)))
     return q_out
+
+
+def mla_absorb_o(o_latent, w_uv, out, stream=None):
+    """out[b,h,:] = w_uv[h] . o_latent[b,h,:] (the output absorption)."""
+    B, H = int(o_latent.shape[0]), int(o_latent.shape[1])
+    _need(o_latent, "o_latent", torch.bfloat16, (B, H, 512))
+    _need(w_uv, "w_uv", torch.bfloat16, (H, 128, 512))
+    _need(out, "out", torch.bfloat16)
+    if out.dim() != 3 or tuple(out.shape[:2]) != (B, H):
+        raise ValueError("out must be [B,H,ldo]")
+    _check("mla_absorb_o", load().mla_absorb_o(_ptr(o_latent), _ptr(w_uv), _ptr(out),
+                                               int(out.shape[2]), B, H, _stream(stream)))
+    return out
 
 
 def mla_absorb_get_error(stream=None) -> int:
@@ -239,6 +254,8 @@ def to_device(w, device="cuda"):
     if w.q_nope is not None:
         d["q_nope"] = w.q_nope.to(device)
         d["w_uk"] = w.w_uk.to(device)
+    if w.w_uv is not None:
+        d["w_uv"] = w.w_uv.to(device)
     return d
 
 

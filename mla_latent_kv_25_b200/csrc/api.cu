@@ -146,6 +146,28 @@ mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, const void* q_ro
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+mla_status_t mla_absorb_o(const void* o_latent, const void* w_uv, void* out, int ldo, int B, int H,
+                          void* stream) {
+  if (!o_latent || !w_uv || !out) return MLA_ERR_INVALID_ARG;
+  if (B < 1 || B > kMaxBatch || !valid_heads(H)) return MLA_ERR_INVALID_ARG;
+  if (ldo < kNope || ldo % 8 != 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o_latent) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
+  CUtensorMap omap, wmap;
+  // o_latent [B, H, 512] as {c, h, b}: one box = 128 batch rows x 64 c of one head
+  const cuuint64_t odims[3] = {cuuint64_t(kDc), cuuint64_t(H), cuuint64_t(B)};
+  const cuuint64_t ostr[2] = {cuuint64_t(kDc) * 2, cuuint64_t(H) * kDc * 2};
+  const cuuint32_t obox[3] = {64, 1, 128};
+  if (!encode_bf16(&omap, o_latent, 3, odims, ostr, obox)) return MLA_ERR_CUDA;
+  // W_UV [H, 128, 512] as rows (h, d) x columns c, one box = the 128 rows of a head
+  const cuuint64_t wdims[2] = {cuuint64_t(kDc), cuuint64_t(H) * kNope};
+  const cuuint64_t wstr[1] = {cuuint64_t(kDc) * 2};
+  const cuuint32_t wbox[2] = {64, 128};
+  if (!encode_bf16(&wmap, w_uv, 2, wdims, wstr, wbox)) return MLA_ERR_CUDA;
+  cudaError_t e = launch_absorb_o(omap, wmap, static_cast<__nv_bfloat16*>(out), ldo, B, H,
+                                  kDefaultSpin, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 mla_status_t mla_absorb_get_error(void* stream, uint32_t* err_bits) {
   if (!err_bits) return MLA_ERR_INVALID_ARG;
   uint32_t v = 0;

@@ -50,7 +50,11 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int B, in
 cudaError_t launch_absorb_q(const CUtensorMap& qmap, const CUtensorMap& wmap,
                             const __nv_bfloat16* q_rope, __nv_bfloat16* q_out, int ldq, int B,
                             int H, long long spin_limit, cudaStream_t stream);
-// Copies the absorption kernel's error word to *bits and clears it (synchronises `stream`).
+// omap: 3-D view {c 512, h H, b B} of o_latent with box {64, 1, 128}; wmap: 2-D
+// view {c 512, rows H*128} of W_UV with box {64, 128}; both 128 B swizzled.
+cudaError_t launch_absorb_o(const CUtensorMap& omap, const CUtensorMap& wmap, __nv_bfloat16* out,
+                            int ldo, int B, int H, long long spin_limit, cudaStream_t stream);
+// Copies the absorption kernels' error word to *bits and clears it (synchronises `stream`).
 cudaError_t absorb_take_error(uint32_t* bits, cudaStream_t stream);
 
 }  // namespace mla

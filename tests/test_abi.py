@@ -90,5 +90,11 @@ def test_absorb_and_combine_reject_invalid_arguments_on_host():
     assert lib.mla_absorb_q(None, g, None, g, 576, 1, 16, None) == 1
     assert lib.mla_absorb_q(g, g, g, g, 512, 1, 16, None) == 1      # ldq too small for q_rope
     assert lib.mla_absorb_q(g, g, None, g, 516, 1, 16, None) == 1   # ldq not a multiple of 8
+    assert lib.mla_absorb_o(None, g, g, 128, 1, 16, None) == 1
+    assert lib.mla_absorb_o(g, g, g, 120, 1, 16, None) == 1       # ldo below 128
+    assert lib.mla_absorb_o(g, g, g, 132, 1, 16, None) == 1       # ldo not a multiple of 8
+    assert lib.mla_absorb_o(g, g, g, 128, 1, 24, None) == 1       # H not a multiple of 16
+    assert lib.mla_absorb_o(g, g, P(4100), 128, 1, 16, None) == 1  # misaligned output
+    assert lib.mla_absorb_get_error(None, None) == 1
     assert lib.mla_combine(None, g, 1, 16, 2, g, g, None) == 1
     assert lib.mla_combine(g, g, 1, 16, 0, g, g, None) == 1

@@ -171,6 +171,42 @@ def test_absorb_q_without_rope_leaves_tail():
     assert torch.all(q_out[:, :, 512:] == 5.0)
 
 
+@pytest.mark.parametrize("B,H,ldo", [(1, 16, 128), (64, 128, 128), (130, 32, 136)])
+def test_absorb_o_matches_oracle(B, H, ldo):
+    """Tensor-core output absorption: several 128-row tiles with a ragged last
+    tile and a padded row stride."""
+    w = inputs.make("v3", B=B, H=H, L=[1] * B, seed=35)
+    g = torch.Generator().manual_seed(36)
+    o = (torch.randn((B, H, 512), generator=g) * 0.05).to(torch.bfloat16)
+    out = torch.full((B, H, ldo), 3.0, dtype=torch.bfloat16, device="cuda")
+    binding.mla_absorb_o(o.cuda(), w.w_uv.cuda(), out)
+    assert binding.mla_absorb_get_error() == 0
+    ref = oracle.absorb_o(o, w.w_uv)
+    assert_close(to_np(out[:, :, :128]).reshape(-1, 128), ref.reshape(-1, 128), "absorb_o")
+    assert torch.all(out[:, :, 128:] == 3.0)
+
+
+def test_decode_then_output_absorption_matches_oracle_chain():
+    """The layer output of the absorbed path: mla_absorb_q -> mla_decode ->
+    mla_absorb_o on the GPU against the oracle's chain on the same inputs."""
+    w = inputs.make("v3", B=3, H=32, L=[300, 64, 129], seed=37, q_std=1.0)
+    d = binding.to_device(w)
+    q = torch.empty((3, 32, 576), dtype=torch.bfloat16, device="cuda")
+    binding.mla_absorb_q(d["q_nope"], d["w_uk"], w.q[:, :, 512:].contiguous().cuda(), q)
+    d["q"] = q
+    out, lse, ws = binding.decode_device(d, w.softmax_scale, num_splits=4)
+    assert binding.mla_get_device_error(ws) == 0
+    o_heads = torch.empty((3, 32, 128), dtype=torch.bfloat16, device="cuda")
+    binding.mla_absorb_o(out, d["w_uv"], o_heads)
+    assert binding.mla_absorb_get_error() == 0
+    # oracle chain on the same bf16 values the GPU consumed at each step
+    w.q = q.cpu()
+    ro, _ = oracle.decode_workload(w)
+    o_bf = torch.from_numpy(ro.reshape(3, 32, 512)).to(torch.bfloat16)
+    ref = oracle.absorb_o(o_bf, w.w_uv)
+    assert_close(to_np(o_heads).reshape(-1, 128), ref.reshape(-1, 128), "decode + absorb_o")
+
+
 # ---------------------------------------------------------------- full-size configs, sampled rows
 
 def _sample_rows(w, n, seed):
