@@ -194,6 +194,47 @@ mla_status_t mla_decode_noalloc(const void *q, mla_cache_dtype_t cache_dtype, co
                                 int num_blocks, int max_blocks_per_seq, float softmax_scale,
                                 void *out, float *lse, int num_splits, void *stream);
 
+/*
+ * mla_cache_append - write the rows of T new tokens into the paged bf16 cache
+ * ("Empirical Gains": only c^KV and the decoupled RoPE key are cached; the key
+ * is rotated before caching, in fp32 — eeumee.net, FP8/FP32 Mixed Precision):
+ *     cache[block_table[b*max_blocks_per_seq + p/64], p%64, :] = [c_kv[t] | RoPE(k_r[t], p)]
+ * with b = seq_idx[t], p = pos[t].  RoPE rotates consecutive pairs
+ * (x_2i, x_2i+1) by p * 10000^(-2i/64).
+ * c_kv: bf16 [T,512] (16-byte aligned); k_r: bf16 [T,64], before rotation;
+ * seq_idx, pos: int32 [T] on the device; block_table: int32 [B, max_blocks_per_seq];
+ * cache: bf16 [num_blocks,64,576] (16-byte aligned).  Tokens with b or p out
+ * of range, or whose block id is out of range, are skipped and recorded as
+ * MLA_DEVERR_SEQ_TOO_LONG / MLA_DEVERR_BAD_BLOCK (mla_cache_get_error).  Two
+ * tokens must not target the same row.  T = 0 is a no-op.
+ */
+mla_status_t mla_cache_append(const void *c_kv, const void *k_r, const int32_t *seq_idx,
+                              const int32_t *pos, int T, const int32_t *block_table, int B,
+                              int max_blocks_per_seq, int num_blocks, void *cache, void *stream);
+
+/*
+ * mla_cache_quantize_fp8 - convert n whole blocks of a bf16 cache to the fp8
+ * layout mla_decode reads (MLA_CACHE_FP8_E4M3), at the same block ids
+ * (eeumee.net, FP8/FP32 Mixed Precision; the per-block scale follows the
+ * E4M3 range): for each listed block k,
+ *     block_scale[k] = amax_k / 448 (1 if the block's c_kv is all zero),
+ *     codes[k, r, c] = E4M3(c_kv[k, r, c] / block_scale[k])  (nearest, saturating),
+ *     k_rope[k, r, :] = cache_bf16[k, r, 512:576]  (copied),
+ * the divisions in IEEE fp32.  cache_bf16: bf16 [num_blocks,64,576];
+ * blocks: int32 [n] on the device; codes: u8 [num_blocks,64,512];
+ * k_rope: bf16 [num_blocks,64,64]; block_scale: f32 [num_blocks].  Ids out of
+ * range are skipped and recorded as MLA_DEVERR_BAD_BLOCK.  n = 0 is a no-op.
+ */
+mla_status_t mla_cache_quantize_fp8(const void *cache_bf16, const int32_t *blocks, int n,
+                                    int num_blocks, void *codes, void *k_rope, float *block_scale,
+                                    void *stream);
+
+/*
+ * mla_cache_get_error - device error bits of the cache writers since the last
+ * call; synchronises `stream` and clears them.
+ */
+mla_status_t mla_cache_get_error(void *stream, uint32_t *err_bits);
+
 /* mla_status_string - a static, human-readable name for a status code. */
 const char *mla_status_string(mla_status_t status);
 

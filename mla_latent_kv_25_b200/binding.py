@@ -29,7 +29,8 @@ DEVERR_SEQ_TOO_LONG = 0x2
 DEVERR_TIMEOUT = 0x4
 
 # every symbol include/mla.h declares
-EXPORTS = ("mla_absorb_q", "mla_absorb_o", "mla_absorb_get_error", "mla_decode_workspace_bytes", "mla_decode",
+EXPORTS = ("mla_absorb_q", "mla_absorb_o", "mla_absorb_get_error", "mla_cache_append",
+           "mla_cache_quantize_fp8", "mla_cache_get_error", "mla_decode_workspace_bytes", "mla_decode",
            "mla_combine", "mla_get_device_error", "mla_status_string", "mla_num_sms",
            "mla_decode_noalloc")
 
@@ -59,6 +60,12 @@ def load():
         L.mla_absorb_q.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
         L.mla_absorb_o.restype = i32
         L.mla_absorb_o.argtypes = [vp, vp, vp, i32, i32, i32, vp]
+        L.mla_cache_append.restype = i32
+        L.mla_cache_append.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp]
+        L.mla_cache_quantize_fp8.restype = i32
+        L.mla_cache_quantize_fp8.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp]
+        L.mla_cache_get_error.restype = i32
+        L.mla_cache_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_absorb_get_error.restype = i32
         L.mla_absorb_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_decode_workspace_bytes.restype = u64
@@ -156,6 +163,42 @@ def mla_absorb_o(o_latent, w_uv, out, stream=None):
     _check("mla_absorb_o", load().mla_absorb_o(_ptr(o_latent), _ptr(w_uv), _ptr(out),
                                                int(out.shape[2]), B, H, _stream(stream)))
     return out
+
+
+def mla_cache_append(c_kv, k_r, seq_idx, pos, block_table, cache, stream=None):
+    """Write [c_kv | RoPE(k_r, pos)] rows of new tokens into the paged bf16 cache."""
+    T = int(c_kv.shape[0])
+    _need(c_kv, "c_kv", torch.bfloat16, (T, 512))
+    _need(k_r, "k_r", torch.bfloat16, (T, 64))
+    _need(seq_idx, "seq_idx", torch.int32, (T,))
+    _need(pos, "pos", torch.int32, (T,))
+    _need(block_table, "block_table", torch.int32)
+    _need(cache, "cache", torch.bfloat16)
+    B, mb = int(block_table.shape[0]), int(block_table.shape[1])
+    _check("mla_cache_append", load().mla_cache_append(
+        _ptr(c_kv), _ptr(k_r), _ptr(seq_idx), _ptr(pos), T, _ptr(block_table), B, mb,
+        int(cache.shape[0]), _ptr(cache), _stream(stream)))
+    return cache
+
+
+def mla_cache_quantize_fp8(cache_bf16, blocks, codes, k_rope, block_scale, stream=None):
+    """Convert the listed blocks of a bf16 cache to the fp8 layout."""
+    _need(cache_bf16, "cache_bf16", torch.bfloat16)
+    _need(blocks, "blocks", torch.int32)
+    _need(codes, "codes", torch.uint8)
+    _need(k_rope, "k_rope", torch.bfloat16)
+    _need(block_scale, "block_scale", torch.float32)
+    _check("mla_cache_quantize_fp8", load().mla_cache_quantize_fp8(
+        _ptr(cache_bf16), _ptr(blocks), int(blocks.numel()), int(cache_bf16.shape[0]), _ptr(codes),
+        _ptr(k_rope), _ptr(block_scale), _stream(stream)))
+    return codes, k_rope, block_scale
+
+
+def mla_cache_get_error(stream=None) -> int:
+    """Synchronise the stream, return and clear the cache writers' error bits."""
+    v = ctypes.c_uint32(0)
+    _check("mla_cache_get_error", load().mla_cache_get_error(_stream(stream), ctypes.byref(v)))
+    return int(v.value)
 
 
 def mla_absorb_get_error(stream=None) -> int:

@@ -168,6 +168,48 @@ mla_status_t mla_absorb_o(const void* o_latent, const void* w_uv, void* out, int
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+mla_status_t mla_cache_append(const void* c_kv, const void* k_r, const int32_t* seq_idx,
+                              const int32_t* pos, int T, const int32_t* block_table, int B,
+                              int max_blocks_per_seq, int num_blocks, void* cache, void* stream) {
+  if (!c_kv || !k_r || !seq_idx || !pos || !block_table || !cache) return MLA_ERR_INVALID_ARG;
+  if (T < 0 || T > kMaxBatch * 64 || B < 1 || B > kMaxBatch) return MLA_ERR_INVALID_ARG;
+  if (num_blocks < 1 || max_blocks_per_seq < 1 || max_blocks_per_seq > (1 << 24)) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(c_kv) || !aligned16(cache) || (reinterpret_cast<uintptr_t>(k_r) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_idx) & 3u) || (reinterpret_cast<uintptr_t>(pos) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u))
+    return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  cudaError_t e = launch_cache_append(static_cast<const __nv_bfloat16*>(c_kv),
+                                      static_cast<const __nv_bfloat16*>(k_r), seq_idx, pos, T,
+                                      block_table, B, max_blocks_per_seq, num_blocks,
+                                      static_cast<__nv_bfloat16*>(cache), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_cache_quantize_fp8(const void* cache_bf16, const int32_t* blocks, int n,
+                                    int num_blocks, void* codes, void* k_rope, float* block_scale,
+                                    void* stream) {
+  if (!cache_bf16 || !blocks || !codes || !k_rope || !block_scale) return MLA_ERR_INVALID_ARG;
+  if (n < 0 || n > (1 << 24) || num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(cache_bf16) || !aligned16(codes) || !aligned16(k_rope) ||
+      (reinterpret_cast<uintptr_t>(blocks) & 3u) || (reinterpret_cast<uintptr_t>(block_scale) & 3u))
+    return MLA_ERR_INVALID_ARG;
+  if (n == 0) return MLA_OK;
+  cudaError_t e = launch_cache_quantize_fp8(static_cast<const __nv_bfloat16*>(cache_bf16), blocks, n,
+                                            num_blocks, static_cast<uint8_t*>(codes),
+                                            static_cast<__nv_bfloat16*>(k_rope), block_scale,
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_cache_get_error(void* stream, uint32_t* err_bits) {
+  if (!err_bits) return MLA_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  if (cache_take_error(&v, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  *err_bits = v;
+  return MLA_OK;
+}
+
 mla_status_t mla_absorb_get_error(void* stream, uint32_t* err_bits) {
   if (!err_bits) return MLA_ERR_INVALID_ARG;
   uint32_t v = 0;

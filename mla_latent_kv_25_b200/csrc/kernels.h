@@ -54,6 +54,15 @@ cudaError_t launch_absorb_q(const CUtensorMap& qmap, const CUtensorMap& wmap,
 // view {c 512, rows H*128} of W_UV with box {64, 128}; both 128 B swizzled.
 cudaError_t launch_absorb_o(const CUtensorMap& omap, const CUtensorMap& wmap, __nv_bfloat16* out,
                             int ldo, int B, int H, long long spin_limit, cudaStream_t stream);
+cudaError_t launch_cache_append(const __nv_bfloat16* c_kv, const __nv_bfloat16* k_r,
+                                const int32_t* seq_idx, const int32_t* pos, int T,
+                                const int32_t* block_table, int B, int max_blocks, int num_blocks,
+                                __nv_bfloat16* cache, cudaStream_t stream);
+cudaError_t launch_cache_quantize_fp8(const __nv_bfloat16* cache_bf16, const int32_t* blocks, int n,
+                                      int num_blocks, uint8_t* codes, __nv_bfloat16* k_rope,
+                                      float* block_scale, cudaStream_t stream);
+// Copies the cache writers' error word to *bits and clears it (synchronises `stream`).
+cudaError_t cache_take_error(uint32_t* bits, cudaStream_t stream);
 // Copies the absorption kernels' error word to *bits and clears it (synchronises `stream`).
 cudaError_t absorb_take_error(uint32_t* bits, cudaStream_t stream);
 

@@ -96,5 +96,13 @@ def test_absorb_and_combine_reject_invalid_arguments_on_host():
     assert lib.mla_absorb_o(g, g, g, 128, 1, 24, None) == 1       # H not a multiple of 16
     assert lib.mla_absorb_o(g, g, P(4100), 128, 1, 16, None) == 1  # misaligned output
     assert lib.mla_absorb_get_error(None, None) == 1
+    assert lib.mla_cache_append(None, g, g, g, 1, g, 1, 1, 1, g, None) == 1
+    assert lib.mla_cache_append(g, g, g, g, -1, g, 1, 1, 1, g, None) == 1   # negative T
+    assert lib.mla_cache_append(P(4100), g, g, g, 1, g, 1, 1, 1, g, None) == 1  # misaligned rows
+    assert lib.mla_cache_append(g, g, g, g, 0, g, 1, 1, 1, g, None) == 0    # T = 0: nothing to do
+    assert lib.mla_cache_quantize_fp8(None, g, 1, 1, g, g, g, None) == 1
+    assert lib.mla_cache_quantize_fp8(g, g, -1, 1, g, g, g, None) == 1      # negative n
+    assert lib.mla_cache_quantize_fp8(g, g, 1, 0, g, g, g, None) == 1       # no blocks
+    assert lib.mla_cache_get_error(None, None) == 1
     assert lib.mla_combine(None, g, 1, 16, 2, g, g, None) == 1
     assert lib.mla_combine(g, g, 1, 16, 0, g, g, None) == 1
