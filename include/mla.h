@@ -235,6 +235,17 @@ mla_status_t mla_cache_quantize_fp8(const void *cache_bf16, const int32_t *block
  */
 mla_status_t mla_cache_get_error(void *stream, uint32_t *err_bits);
 
+/*
+ * mla_set_wait_limit - bound, in SM clock cycles, of every wait inside the
+ * decode kernels launched from now on (process-wide; default about two
+ * seconds of SM clock; cycles <= 0 restores the default).  Returns the
+ * previous bound.  A wait that reaches the bound records MLA_DEVERR_TIMEOUT,
+ * makes every role of the kernel leave its loop, lets copies in flight land
+ * and exits; the outputs of that launch are then undefined, the context stays
+ * usable.  Meant for tests of that failure path and for diagnosis.
+ */
+long long mla_set_wait_limit(long long cycles);
+
 /* mla_status_string - a static, human-readable name for a status code. */
 const char *mla_status_string(mla_status_t status);
 

@@ -30,7 +30,7 @@ DEVERR_TIMEOUT = 0x4
 
 # every symbol include/mla.h declares
 EXPORTS = ("mla_absorb_q", "mla_absorb_o", "mla_absorb_get_error", "mla_cache_append",
-           "mla_cache_quantize_fp8", "mla_cache_get_error", "mla_decode_workspace_bytes", "mla_decode",
+           "mla_cache_quantize_fp8", "mla_cache_get_error", "mla_set_wait_limit", "mla_decode_workspace_bytes", "mla_decode",
            "mla_combine", "mla_get_device_error", "mla_status_string", "mla_num_sms",
            "mla_decode_noalloc")
 
@@ -60,6 +60,8 @@ def load():
         L.mla_absorb_q.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
         L.mla_absorb_o.restype = i32
         L.mla_absorb_o.argtypes = [vp, vp, vp, i32, i32, i32, vp]
+        L.mla_set_wait_limit.restype = ctypes.c_longlong
+        L.mla_set_wait_limit.argtypes = [ctypes.c_longlong]
         L.mla_cache_append.restype = i32
         L.mla_cache_append.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp]
         L.mla_cache_quantize_fp8.restype = i32
@@ -192,6 +194,12 @@ def mla_cache_quantize_fp8(cache_bf16, blocks, codes, k_rope, block_scale, strea
         _ptr(cache_bf16), _ptr(blocks), int(blocks.numel()), int(cache_bf16.shape[0]), _ptr(codes),
         _ptr(k_rope), _ptr(block_scale), _stream(stream)))
     return codes, k_rope, block_scale
+
+
+def mla_set_wait_limit(cycles: int) -> int:
+    """Bound of the decode kernels' waits in SM cycles (<= 0: the default);
+    returns the previous bound."""
+    return int(load().mla_set_wait_limit(int(cycles)))
 
 
 def mla_cache_get_error(stream=None) -> int:

@@ -2,6 +2,7 @@
 // workspace layout, choice of the split-KV engine count, and the launches.
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/mla.h"
@@ -96,6 +97,7 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
 constexpr int kMaxSplits = 4096;
 constexpr int kMaxBatch = 1 << 20;
 constexpr long long kDefaultSpin = 4000000000LL;  // ~2 s of SM clock
+std::atomic<long long> g_decode_wait_limit{kDefaultSpin};  // set by mla_set_wait_limit
 
 bool valid_heads(int H) { return H >= 16 && H <= kMaxHeads && H % 16 == 0; }
 
@@ -116,6 +118,11 @@ const char* mla_status_string(mla_status_t s) {
 }
 
 int mla_num_sms(void) { return device_sms(); }
+
+long long mla_set_wait_limit(long long cycles) {
+  const long long v = cycles > 0 ? cycles : kDefaultSpin;
+  return g_decode_wait_limit.exchange(v);
+}
 
 size_t mla_decode_workspace_bytes(int B, int H, int num_splits) {
   if (B < 1 || B > kMaxBatch || !valid_heads(H) || num_splits < 0 || num_splits > kMaxSplits)
@@ -265,7 +272,7 @@ mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void
   p.lse_part = reinterpret_cast<float*>(wsb + ws.lse_part);
   p.o_part = reinterpret_cast<float*>(wsb + ws.o_part);
   p.P = P;
-  p.spin_limit = kDefaultSpin;
+  p.spin_limit = g_decode_wait_limit.load();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   cudaError_t e;
