@@ -147,6 +147,26 @@ mla_status_t mla_decode(const void *q, mla_cache_dtype_t cache_dtype, const void
                         int num_splits, void *stream);
 
 /*
+ * mla_decode_multi - decode q_len query tokens per sequence at once (multi-
+ * token prediction / speculative drafts): the q_len * H query rows of a
+ * sequence share every cache row they read, so one pass over the cache serves
+ * them all.  Token j of sequence b is the (seq_lens[b] - q_len + 1 + j)-th
+ * token: it attends to the first seq_lens[b] - (q_len - 1 - j) cached tokens
+ * (the drafts' own rows are already in the cache; causal among the drafts).
+ * q: bf16 [B, q_len, H, 576]; out: bf16 [B, q_len, H, 512]; lse: f32
+ * [B, q_len, H]; bf16 cache only (the fp8 cache returns MLA_ERR_UNSUPPORTED
+ * for q_len > 1).  q_len * H must be a multiple of 16 and at most 128.
+ * workspace: mla_decode_workspace_bytes(B, q_len * H, num_splits) bytes.
+ * Other arguments and error behaviour as mla_decode; a token that sees no
+ * cached token gives out = 0 and lse = -inf.
+ */
+mla_status_t mla_decode_multi(const void *q, int q_len, const void *cache,
+                              const int32_t *block_table, const int32_t *seq_lens, int B, int H,
+                              int num_blocks, int max_blocks_per_seq, float softmax_scale,
+                              void *out, float *lse, void *workspace, size_t workspace_bytes,
+                              int num_splits, void *stream);
+
+/*
  * mla_combine - log-sum-exp merge of S split-KV partial results (the
  * flash-decoding merge that makes split-KV equal the unsplit softmax):
  *     M = max_i lse_part[r,i];  lse[r] = M + log sum_i exp(lse_part[r,i] - M)

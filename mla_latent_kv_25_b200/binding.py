@@ -30,7 +30,7 @@ DEVERR_TIMEOUT = 0x4
 
 # every symbol include/mla.h declares
 EXPORTS = ("mla_absorb_q", "mla_absorb_o", "mla_absorb_get_error", "mla_cache_append",
-           "mla_cache_quantize_fp8", "mla_cache_get_error", "mla_set_wait_limit", "mla_decode_workspace_bytes", "mla_decode",
+           "mla_cache_quantize_fp8", "mla_cache_get_error", "mla_set_wait_limit", "mla_decode_multi", "mla_decode_workspace_bytes", "mla_decode",
            "mla_combine", "mla_get_device_error", "mla_status_string", "mla_num_sms",
            "mla_decode_noalloc")
 
@@ -60,6 +60,9 @@ def load():
         L.mla_absorb_q.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
         L.mla_absorb_o.restype = i32
         L.mla_absorb_o.argtypes = [vp, vp, vp, i32, i32, i32, vp]
+        L.mla_decode_multi.restype = i32
+        L.mla_decode_multi.argtypes = [vp, i32, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, vp, vp,
+                                       vp, u64, i32, vp]
         L.mla_set_wait_limit.restype = ctypes.c_longlong
         L.mla_set_wait_limit.argtypes = [ctypes.c_longlong]
         L.mla_cache_append.restype = i32
@@ -194,6 +197,24 @@ def mla_cache_quantize_fp8(cache_bf16, blocks, codes, k_rope, block_scale, strea
         _ptr(cache_bf16), _ptr(blocks), int(blocks.numel()), int(cache_bf16.shape[0]), _ptr(codes),
         _ptr(k_rope), _ptr(block_scale), _stream(stream)))
     return codes, k_rope, block_scale
+
+
+def mla_decode_multi(q, cache, block_table, seq_lens, softmax_scale, out, lse, workspace, *,
+                     num_splits=0, stream=None):
+    """Decode q_len query tokens per sequence (q [B,q_len,H,576], bf16 cache)."""
+    B, q_len, H = int(q.shape[0]), int(q.shape[1]), int(q.shape[2])
+    _need(q, "q", torch.bfloat16, (B, q_len, H, 576))
+    _need(cache, "cache", torch.bfloat16)
+    _need(block_table, "block_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    _need(out, "out", torch.bfloat16, (B, q_len, H, 512))
+    _need(lse, "lse", torch.float32, (B, q_len, H))
+    _need(workspace, "workspace", torch.uint8)
+    _check("mla_decode_multi", load().mla_decode_multi(
+        _ptr(q), q_len, _ptr(cache), _ptr(block_table), _ptr(seq_lens), B, H, int(cache.shape[0]),
+        int(block_table.shape[1]), float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+        int(workspace.numel()), int(num_splits), _stream(stream)))
+    return out, lse
 
 
 def mla_set_wait_limit(cycles: int) -> int:

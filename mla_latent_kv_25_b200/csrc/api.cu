@@ -225,14 +225,23 @@ mla_status_t mla_absorb_get_error(void* stream, uint32_t* err_bits) {
   return MLA_OK;
 }
 
-mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void* cache,
-                        const void* k_rope, const float* block_scale, const int32_t* block_table,
-                        const int32_t* seq_lens, int B, int H, int num_blocks,
-                        int max_blocks_per_seq, float softmax_scale, void* out, float* lse,
-                        void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by mla_decode (q_len = 1) and mla_decode_multi: the q_len query
+// tokens of a sequence are q_len * H rows of one engine's contraction.
+mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype, const void* cache,
+                         const void* k_rope, const float* block_scale, const int32_t* block_table,
+                         const int32_t* seq_lens, int B, int H, int num_blocks,
+                         int max_blocks_per_seq, float softmax_scale, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
   if (!q || !cache || !block_table || !seq_lens || !out || !lse || !workspace)
     return MLA_ERR_INVALID_ARG;
-  if (B < 1 || B > kMaxBatch || !valid_heads(H)) return MLA_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > kMaxHeads / 16 || H < 1) return MLA_ERR_INVALID_ARG;
+  const int rows = H * q_len;
+  if (B < 1 || B > kMaxBatch || !valid_heads(rows)) return MLA_ERR_INVALID_ARG;
+  if (q_len > 1 && cache_dtype == MLA_CACHE_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
   if (num_blocks < 1 || max_blocks_per_seq < 1 || max_blocks_per_seq > (1 << 24))
     return MLA_ERR_INVALID_ARG;
   if (num_splits < 0 || num_splits > kMaxSplits) return MLA_ERR_INVALID_ARG;
@@ -249,7 +258,7 @@ mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void
     return MLA_ERR_INVALID_ARG;
   const int P = resolve_engines(num_splits, B);
   if (P < 1) return MLA_ERR_CUDA;
-  const WsLayout ws = ws_layout(B, H, P);
+  const WsLayout ws = ws_layout(B, rows, P);
   if (workspace_bytes < ws.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
 
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
@@ -261,7 +270,9 @@ mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.B = B;
-  p.H = H;
+  p.H = rows;
+  p.q_len = q_len;
+  p.h_per_q = H;
   p.num_blocks = num_blocks;
   p.max_blocks = max_blocks_per_seq;
   p.softmax_scale = softmax_scale;
@@ -285,9 +296,32 @@ mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void
     e = launch_decode_simt(p, fp8, st);
   }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
-  e = launch_merge_pieces(seq_lens, B, max_blocks_per_seq, H, p.seq_info, p.lse_part, p.o_part,
+  e = launch_merge_pieces(seq_lens, B, max_blocks_per_seq, rows, p.seq_info, p.lse_part, p.o_part,
                           p.out, p.lse, p.err, st);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status_t mla_decode(const void* q, mla_cache_dtype_t cache_dtype, const void* cache,
+                        const void* k_rope, const float* block_scale, const int32_t* block_table,
+                        const int32_t* seq_lens, int B, int H, int num_blocks,
+                        int max_blocks_per_seq, float softmax_scale, void* out, float* lse,
+                        void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
+  return decode_rows(q, 1, cache_dtype, cache, k_rope, block_scale, block_table, seq_lens, B, H,
+                     num_blocks, max_blocks_per_seq, softmax_scale, out, lse, workspace,
+                     workspace_bytes, num_splits, stream);
+}
+
+mla_status_t mla_decode_multi(const void* q, int q_len, const void* cache, const int32_t* block_table,
+                              const int32_t* seq_lens, int B, int H, int num_blocks,
+                              int max_blocks_per_seq, float softmax_scale, void* out, float* lse,
+                              void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
+  return decode_rows(q, q_len, MLA_CACHE_BF16, cache, nullptr, nullptr, block_table, seq_lens, B, H,
+                     num_blocks, max_blocks_per_seq, softmax_scale, out, lse, workspace,
+                     workspace_bytes, num_splits, stream);
 }
 
 mla_status_t mla_combine(const float* o_part, const float* lse_part, int B, int H, int S,

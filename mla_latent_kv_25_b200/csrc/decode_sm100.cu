@@ -401,6 +401,10 @@ __device__ void score_softmax(const Ctx& c) {
     if (w.b < w.B && w.pre < w.e) prefetch_q_rows_l2(p, w.b, h);  // next segment's query
 
     SoftmaxState st{-INFINITY, 0.f};
+    // multi-token decode: this row's query token sees the sequence without
+    // its last `short_by` tokens (0 for a plain decode)
+    const int short_by = h < p.H ? p.q_len - 1 - h / p.h_per_q : 0;
+    const int row_len = g.len - short_by;
     // one block per iteration (a single inlined copy of softmax_block); the
     // blocks of a pass share one S buffer, released after its last read
     for (int j = g.blk_lo; j < g.blk_hi; ++j) {
@@ -426,7 +430,8 @@ __device__ void score_softmax(const Ctx& c) {
         mbar_arrive(bar_addr(c.bars->s_empty[sb]));
         ++pit;
       }
-      if (!softmax_block(c, sv, nv, j == g.blk_lo, sl2, pos, st, it, h, q4)) {
+      const int nv_row = max(0, min(nv, row_len - j * kBlock));
+      if (!softmax_block(c, sv, nv_row, j == g.blk_lo, sl2, pos, st, it, h, q4)) {
         alive = false;
         break;
       }

@@ -9,7 +9,7 @@
 namespace mla {
 
 struct DecodeParams {
-  const __nv_bfloat16* q;          // [B,H,576]
+  const __nv_bfloat16* q;          // [B,H,576] (H = rows per sequence)
   const void* cache;               // bf16 [NB,64,576] | u8 [NB,64,512]
   const __nv_bfloat16* k_rope;     // fp8 cache: [NB,64,64]
   const float* block_scale;        // fp8 cache: [NB]
@@ -25,6 +25,10 @@ struct DecodeParams {
   float* o_part;                   // [2P,H,512]
   int P;                           // number of split-KV engines
   long long spin_limit;            // bounded-wait limit (clock64 cycles)
+  // Multi-token decode: the H rows of a sequence are q_len query tokens of
+  // h_per_q heads each (row r = token r / h_per_q); token j sees the
+  // sequence without its last q_len - 1 - j tokens.  q_len = 1: plain decode.
+  int q_len, h_per_q;
 };
 
 // CUDA-core decode (any H multiple of 16); fp8: cache is E4M3.

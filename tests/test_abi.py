@@ -104,5 +104,10 @@ def test_absorb_and_combine_reject_invalid_arguments_on_host():
     assert lib.mla_cache_quantize_fp8(g, g, -1, 1, g, g, g, None) == 1      # negative n
     assert lib.mla_cache_quantize_fp8(g, g, 1, 0, g, g, g, None) == 1       # no blocks
     assert lib.mla_cache_get_error(None, None) == 1
+    # multi-token decode: q_len * H must be a multiple of 16 and at most 128
+    assert lib.mla_decode_multi(g, 0, g, g, g, 1, 16, 1, 1, 0.1, g, g, g, 1 << 20, 0, None) == 1
+    assert lib.mla_decode_multi(g, 3, g, g, g, 1, 8, 1, 1, 0.1, g, g, g, 1 << 20, 0, None) == 1
+    assert lib.mla_decode_multi(g, 2, g, g, g, 1, 128, 1, 1, 0.1, g, g, g, 1 << 20, 0, None) == 1
+    assert lib.mla_decode_multi(None, 2, g, g, g, 1, 16, 1, 1, 0.1, g, g, g, 1 << 20, 0, None) == 1
     assert lib.mla_combine(None, g, 1, 16, 2, g, g, None) == 1
     assert lib.mla_combine(g, g, 1, 16, 0, g, g, None) == 1

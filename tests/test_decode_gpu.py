@@ -207,6 +207,41 @@ def test_decode_then_output_absorption_matches_oracle_chain():
     assert_close(to_np(o_heads).reshape(-1, 128), ref.reshape(-1, 128), "decode + absorb_o")
 
 
+def _multi_reference(w, q_len, H):
+    """Oracle view of a multi-token decode: token j of sequence b is its own
+    sequence sharing b's block table, shorter by q_len - 1 - j tokens."""
+    B = w.B
+    q = w.q.reshape(B * q_len, H, 576)
+    table = w.block_table.repeat_interleave(q_len, dim=0)
+    lens = torch.tensor([max(0, int(w.seq_lens[b]) - (q_len - 1 - j)) for b in range(B) for j in range(q_len)],
+                        dtype=torch.int32)
+    return oracle.decode_units(q=q, cache=w.cache, block_table=table, seq_lens=lens,
+                               num_blocks=w.num_blocks, softmax_scale=w.softmax_scale,
+                               units=oracle.all_units(B * q_len, H), cache_kind=w.cache_dtype)
+
+
+@pytest.mark.parametrize("q_len,H,num_splits", [(2, 32, 0), (2, 64, 5), (4, 32, 3), (4, 16, 0)])
+def test_multi_token_decode_matches_oracle(q_len, H, num_splits):
+    """q_len query tokens per sequence share the cache pass; token j is causal
+    among the drafts (sees all but the last q_len - 1 - j tokens).  Lengths
+    include one shorter than q_len (its first tokens see nothing)."""
+    B = 4
+    w = inputs.make("v3", B=B, H=q_len * H, L=[700, 65, 130, 2], seed=46, q_std=2.0)
+    d = binding.to_device(w)
+    q = d["q"].reshape(B, q_len, H, 576)
+    out = torch.empty((B, q_len, H, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, q_len, H), dtype=torch.float32, device="cuda")
+    ws = binding.alloc_workspace(B, q_len * H, num_splits)
+    binding.mla_decode_multi(q, d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale, out, lse,
+                             ws, num_splits=num_splits)
+    assert binding.mla_get_device_error(ws) == 0
+    ro, rl = _multi_reference(w, q_len, H)
+    assert_close(to_np(out).reshape(-1, 512), ro, f"multi q_len={q_len}")
+    finite = np.isfinite(rl)
+    assert np.array_equal(np.isfinite(to_np(lse).reshape(-1)), finite)
+    assert_close(to_np(lse).reshape(-1)[finite], rl[finite], f"multi lse q_len={q_len}")
+
+
 # ---------------------------------------------------------------- full-size configs, sampled rows
 
 def _sample_rows(w, n, seed):
