@@ -310,6 +310,30 @@ def run_ours(args, world, rank, local):
     absorb_o_ms = a0.elapsed_time(a1) / K3
     if binding.mla_absorb_get_error(stream) != 0:
         raise RuntimeError("device error in the output absorption")
+
+    # multi-token decode, timed on its own: the same query rows regrouped as
+    # 2 tokens x H/2 heads per sequence (drafts causal among themselves)
+    multi = None
+    if H % 32 == 0:
+        q2 = q.view(B, 2, H // 2, 576)
+        out2 = torch.empty((B, 2, H // 2, 512), dtype=torch.bfloat16, device=dev)
+        lse2 = torch.empty((B, 2, H // 2), dtype=torch.float32, device=dev)
+        ws2 = binding.alloc_workspace(B, H, args.num_splits, device=dev)
+        for _ in range(3):
+            binding.mla_decode_multi(q2, d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale,
+                                     out2, lse2, ws2, num_splits=args.num_splits, stream=stream)
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        K4 = 50
+        m0.record(stream)
+        for _ in range(K4):
+            binding.mla_decode_multi(q2, d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale,
+                                     out2, lse2, ws2, num_splits=args.num_splits, stream=stream)
+        m1.record(stream)
+        torch.cuda.synchronize(dev)
+        if binding.mla_get_device_error(ws2, stream) != 0:
+            raise RuntimeError("device error in the multi-token decode")
+        multi = {"q_len": 2, "heads": H // 2, "ms_per_launch": round(m0.elapsed_time(m1) / K4, 5)}
     if binding.mla_get_device_error(ws, stream) != 0:
         raise RuntimeError("device error during timing")
 
@@ -369,6 +393,9 @@ def run_ours(args, world, rank, local):
                     "d2h_bytes_per_step": int(h_out.numel() * 2 + h_lse.numel() * 4)},
             "gpu_launches": 3 * K,
             "absorb_o": absorb_o_line(B, H, absorb_o_ms, hbm),
+            "multi_token": None if multi is None else dict(
+                multi, algorithmic_bytes=dec_b,
+                frac=round(dec_b / (multi["ms_per_launch"] * 1e-3) / 1e9 / hbm, 4)),
             "clocks": clk,
         }
     if world > 1:
