@@ -430,7 +430,7 @@ __device__ void score_softmax(const Ctx& c) {
         mbar_arrive(bar_addr(c.bars->s_empty[sb]));
         ++pit;
       }
-      const int nv_row = max(0, min(nv, row_len - j * kBlock));
+      const int nv_row = p.q_len > 1 ? max(0, min(nv, row_len - j * kBlock)) : nv;
       if (!softmax_block(c, sv, nv_row, j == g.blk_lo, sl2, pos, st, it, h, q4)) {
         alive = false;
         break;

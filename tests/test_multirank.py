@@ -72,13 +72,14 @@ def test_job_rate_counts_every_rank():
     assert bench.job_rate(1e9, 1, 1000.0) == pytest.approx(1.0)
 
 
-def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
+def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero(tmp_path):
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
            "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
            "--cpu-seconds", "0.3", "--workload", "tiny"]
-    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    env = dict(os.environ, TMPDIR=str(tmp_path))  # torchrun's scratch files go to pytest's tmp dir
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1
