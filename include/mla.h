@@ -105,6 +105,17 @@ mla_status_t mla_absorb_get_error(void *stream, uint32_t *err_bits);
 size_t mla_decode_workspace_bytes(int B, int H, int num_splits);
 
 /*
+ * mla_decode_fp8_workspace_bytes - workspace bytes that let mla_decode run an
+ * fp8 cache on the tensor cores: mla_decode_workspace_bytes(B, H, num_splits)
+ * rounded up to 256, plus a scratch block table (4 * B * max_blocks_per_seq
+ * bytes, rounded up to 256) and a widened bf16 copy of the blocks the batch
+ * reads (73,728 bytes per table entry: B * max_blocks_per_seq blocks of
+ * 64 x 576 bf16).  Returns 0 on invalid arguments or when
+ * B * max_blocks_per_seq exceeds 2^24.
+ */
+size_t mla_decode_fp8_workspace_bytes(int B, int H, int max_blocks_per_seq, int num_splits);
+
+/*
  * mla_decode - the decode-step attention over the paged latent cache
  * ("Empirical Gains": the cache holds only c^KV and the decoupled RoPE key;
  * "The Memory Wall": the whole cache is streamed from HBM every step).
@@ -115,6 +126,15 @@ size_t mla_decode_workspace_bytes(int B, int H, int num_splits);
  * k_rope:      fp8 cache only: bf16 [num_blocks,64,64]; must be NULL for bf16.
  * block_scale: fp8 cache only: f32 [num_blocks], c_kv = e4m3(code) * scale;
  *              must be NULL for bf16.
+ *              The fp8 cache is decoded one of two ways, chosen by
+ *              workspace_bytes.  With at least
+ *              mla_decode_fp8_workspace_bytes(B, H, max_blocks_per_seq,
+ *              num_splits) bytes, a first kernel writes the rows the batch
+ *              reads as bf16 [bf16(e4m3(code) * scale) | k_rope] into the
+ *              workspace (round to nearest even: relative error <= 2^-9 per
+ *              element), and the tensor-core decode reads them.  With less
+ *              (but at least mla_decode_workspace_bytes), a CUDA-core decode
+ *              reads the codes directly, in fp32, about 20x slower.
  * block_table: int32 [B, max_blocks_per_seq]; logical block j of sequence b is
  *              physical block block_table[b*max_blocks_per_seq + j].  Entries
  *              at j >= ceil(seq_lens[b]/64) are never read (pad with -1).
@@ -124,7 +144,7 @@ size_t mla_decode_workspace_bytes(int B, int H, int num_splits);
  * lse:         f32 [B,H], natural log of sum_t exp(score); a sequence of
  *              length 0 gives out = 0 and lse = -inf.
  * workspace:   device buffer of >= mla_decode_workspace_bytes(B,H,num_splits)
- *              bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE; the
+ *              bytes (fp8 cache: see block_scale), 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE; the
  *              library keeps its error word zero except when it records an
  *              error.  One workspace must not be shared by calls that may run
  *              at the same time.
@@ -206,7 +226,9 @@ mla_status_t mla_get_device_error(void *workspace, void *stream, uint32_t *err_b
  * All calls on a device share the array and it keeps the last call's
  * contents: calls that overlap on the GPU race, so serialise them.  Nothing
  * in it needs clearing between calls.  Device-side error bits are recorded
- * in the array but not reported.  Allocates and frees no device memory.
+ * in the array but not reported.  An fp8 cache takes the tensor-core route
+ * when mla_decode_fp8_workspace_bytes(...) fits in the 40 MiB, else the
+ * CUDA-core decode (see mla_decode).  Allocates and frees no device memory.
  */
 mla_status_t mla_decode_noalloc(const void *q, mla_cache_dtype_t cache_dtype, const void *cache,
                                 const void *k_rope, const float *block_scale,

@@ -30,7 +30,8 @@ DEVERR_TIMEOUT = 0x4
 
 # every symbol include/mla.h declares
 EXPORTS = ("mla_absorb_q", "mla_absorb_o", "mla_absorb_get_error", "mla_cache_append",
-           "mla_cache_quantize_fp8", "mla_cache_get_error", "mla_set_wait_limit", "mla_decode_multi", "mla_decode_workspace_bytes", "mla_decode",
+           "mla_cache_quantize_fp8", "mla_cache_get_error", "mla_set_wait_limit", "mla_decode_multi",
+           "mla_decode_workspace_bytes", "mla_decode_fp8_workspace_bytes", "mla_decode",
            "mla_combine", "mla_get_device_error", "mla_status_string", "mla_num_sms",
            "mla_decode_noalloc")
 
@@ -75,6 +76,8 @@ def load():
         L.mla_absorb_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_decode_workspace_bytes.restype = u64
         L.mla_decode_workspace_bytes.argtypes = [i32, i32, i32]
+        L.mla_decode_fp8_workspace_bytes.restype = u64
+        L.mla_decode_fp8_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.mla_decode.restype = i32
         L.mla_decode.argtypes = [vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
                                  vp, vp, vp, u64, i32, vp]
@@ -133,11 +136,24 @@ def mla_decode_workspace_bytes(B: int, H: int, num_splits: int = 0) -> int:
     return int(load().mla_decode_workspace_bytes(int(B), int(H), int(num_splits)))
 
 
-def alloc_workspace(B: int, H: int, num_splits: int = 0, device=None) -> torch.Tensor:
-    """Zero-filled device workspace of the size mla_decode needs."""
-    n = mla_decode_workspace_bytes(B, H, num_splits)
+def mla_decode_fp8_workspace_bytes(B: int, H: int, max_blocks: int, num_splits: int = 0) -> int:
+    return int(load().mla_decode_fp8_workspace_bytes(int(B), int(H), int(max_blocks),
+                                                     int(num_splits)))
+
+
+def alloc_workspace(B: int, H: int, num_splits: int = 0, device=None,
+                    fp8_max_blocks: int | None = None) -> torch.Tensor:
+    """Zero-filled device workspace of the size mla_decode needs.  With
+    ``fp8_max_blocks`` (the block table's width) it also holds the widened
+    bf16 copy that runs an fp8 cache on the tensor cores."""
+    if fp8_max_blocks is None:
+        n = mla_decode_workspace_bytes(B, H, num_splits)
+        fn = "mla_decode_workspace_bytes"
+    else:
+        n = mla_decode_fp8_workspace_bytes(B, H, fp8_max_blocks, num_splits)
+        fn = "mla_decode_fp8_workspace_bytes"
     if n == 0:
-        raise MLAError("mla_decode_workspace_bytes", 1)
+        raise MLAError(fn, 1)
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
@@ -332,13 +348,17 @@ def to_device(w, device="cuda"):
 
 
 def decode_device(d, softmax_scale, num_splits=0, workspace=None, stream=None):
-    """mla_decode on device tensors from ``to_device``; allocates outputs."""
+    """mla_decode on device tensors from ``to_device``; allocates outputs and,
+    unless one is given, the workspace (for an fp8 cache, with room for the
+    widened copy, so that it runs on the tensor cores)."""
     B, H = int(d["q"].shape[0]), int(d["q"].shape[1])
     dev = d["q"].device
     out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, H), dtype=torch.float32, device=dev)
     if workspace is None:
-        workspace = alloc_workspace(B, H, num_splits, device=dev)
+        fp8 = d["cache"].dtype == torch.uint8
+        workspace = alloc_workspace(B, H, num_splits, device=dev,
+                                    fp8_max_blocks=int(d["block_table"].shape[1]) if fp8 else None)
     mla_decode(d["q"], d["cache"], d["block_table"], d["seq_lens"], softmax_scale, out, lse,
                workspace, k_rope=d["k_rope"], block_scale=d["block_scale"],
                num_splits=num_splits, stream=stream)

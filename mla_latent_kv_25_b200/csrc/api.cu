@@ -101,6 +101,25 @@ std::atomic<long long> g_decode_wait_limit{kDefaultSpin};  // set by mla_set_wai
 
 bool valid_heads(int H) { return H >= 16 && H <= kMaxHeads && H % 16 == 0; }
 
+// The fp8 cache's widened bf16 copy, placed after the split-KV workspace:
+// a scratch block table int32 [B * max_blocks] and a dense bf16 cache
+// [B * max_blocks, 64, 576] (block b * max_blocks + j holds logical block j
+// of sequence b).  Its block ids and TMA row coordinates must fit int32.
+constexpr long long kMaxWideBlocks = 1LL << 24;
+
+struct WideLayout {
+  size_t table, cache, total;
+};
+
+WideLayout wide_layout(size_t split_ws_total, int B, int max_blocks) {
+  const size_t n = size_t(B) * size_t(max_blocks);
+  WideLayout w;
+  w.table = align256(split_ws_total);
+  w.cache = align256(w.table + n * 4);
+  w.total = w.cache + n * kBlock * kRow * 2;
+  return w;
+}
+
 }  // namespace
 
 extern "C" {
@@ -130,6 +149,14 @@ size_t mla_decode_workspace_bytes(int B, int H, int num_splits) {
   int P = resolve_engines(num_splits, B);
   if (P < 1) return 0;
   return ws_layout(B, H, P).total;
+}
+
+size_t mla_decode_fp8_workspace_bytes(int B, int H, int max_blocks_per_seq, int num_splits) {
+  if (max_blocks_per_seq < 1 || max_blocks_per_seq > (1 << 24)) return 0;
+  const size_t base = mla_decode_workspace_bytes(B, H, num_splits);
+  if (base == 0) return 0;
+  if (static_cast<long long>(B) * max_blocks_per_seq > kMaxWideBlocks) return 0;
+  return wide_layout(base, B, max_blocks_per_seq).total;
 }
 
 mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, const void* q_rope, void* q_out,
@@ -287,9 +314,27 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   cudaError_t e;
-  if (!fp8) {
+  // The fp8 cache takes the tensor-core decode through its widened bf16 copy
+  // when the workspace has room for it, else the CUDA-core decode.
+  const long long wide_blocks = static_cast<long long>(B) * max_blocks_per_seq;
+  const WideLayout wide = wide_layout(ws.total, B, max_blocks_per_seq);
+  const bool widen = fp8 && wide_blocks <= kMaxWideBlocks && workspace_bytes >= wide.total;
+  if (widen) {
+    int32_t* wide_table = reinterpret_cast<int32_t*>(wsb + wide.table);
+    __nv_bfloat16* wide_cache = reinterpret_cast<__nv_bfloat16*>(wsb + wide.cache);
+    e = launch_fp8_widen(static_cast<const uint8_t*>(cache), p.k_rope, block_scale, block_table,
+                         seq_lens, B, max_blocks_per_seq, num_blocks, wide_table, wide_cache, p.err,
+                         device_sms(), st);
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
+    p.cache = wide_cache;
+    p.k_rope = nullptr;
+    p.block_scale = nullptr;
+    p.block_table = wide_table;
+    p.num_blocks = static_cast<int>(wide_blocks);
+  }
+  if (!fp8 || widen) {
     CUtensorMap tmap;
-    if (!encode_bf16_map(&tmap, cache, uint64_t(num_blocks) * kBlock, kRow, kRow * 2))
+    if (!encode_bf16_map(&tmap, p.cache, uint64_t(p.num_blocks) * kBlock, kRow, kRow * 2))
       return MLA_ERR_CUDA;
     e = launch_decode_sm100(p, tmap, st);
   } else {

@@ -31,7 +31,8 @@ struct DecodeParams {
   int q_len, h_per_q;
 };
 
-// CUDA-core decode (any H multiple of 16); fp8: cache is E4M3.
+// CUDA-core decode (any H multiple of 16); fp8: cache is E4M3.  Used for the
+// fp8 cache when the workspace has no room for the widened bf16 copy.
 cudaError_t launch_decode_simt(const DecodeParams& p, bool fp8, cudaStream_t stream);
 
 // Tensor-core decode (bf16 cache): clusters of two CTAs, one engine each.
@@ -65,6 +66,16 @@ cudaError_t launch_cache_append(const __nv_bfloat16* c_kv, const __nv_bfloat16* 
 cudaError_t launch_cache_quantize_fp8(const __nv_bfloat16* cache_bf16, const int32_t* blocks, int n,
                                       int num_blocks, uint8_t* codes, __nv_bfloat16* k_rope,
                                       float* block_scale, cudaStream_t stream);
+// Widens the fp8 blocks a batch reads into bf16 rows of a dense scratch cache:
+// table entry e = b * max_blocks + j -> wide_table[e] = e and rows
+// wide_cache[e, r, :] = [bf16(e4m3(code) * scale) | k_rope] for r below the
+// sequence length; wide_table[e] = -1 for unread entries and bad block ids
+// (the latter also set kErrBadBlock in *err).
+cudaError_t launch_fp8_widen(const uint8_t* codes, const __nv_bfloat16* k_rope,
+                             const float* block_scale, const int32_t* block_table,
+                             const int32_t* seq_lens, int B, int max_blocks, int num_blocks,
+                             int32_t* wide_table, __nv_bfloat16* wide_cache, uint32_t* err,
+                             int num_sms, cudaStream_t stream);
 // Copies the cache writers' error word to *bits and clears it (synchronises `stream`).
 cudaError_t cache_take_error(uint32_t* bits, cudaStream_t stream);
 // Copies the absorption kernels' error word to *bits and clears it (synchronises `stream`).

@@ -26,6 +26,9 @@
 //     same call.  The array starts zeroed when the library is loaded; its
 //     error word accumulates device-side error bits of all calls and is not
 //     reported by this entry point (invalid block ids are still skipped).
+//   - An fp8 cache runs on the tensor cores (through its widened bf16 copy)
+//     when mla_decode_fp8_workspace_bytes fits in the array, else on the
+//     CUDA-core decode.
 //   - No device memory is allocated or freed by this entry point.
 #include <mutex>
 

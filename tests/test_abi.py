@@ -52,6 +52,21 @@ def test_workspace_size_and_validation_without_device():
     assert lib.mla_decode_workspace_bytes(1, 128, -1) == 0
 
 
+def test_fp8_workspace_adds_the_widened_copy():
+    """The tensor-core route of the fp8 cache needs the split-KV workspace,
+    then a scratch block table (int32 per table entry) and one bf16 block of
+    64 x 576 per table entry, each region 256-byte aligned."""
+    lib = binding.load()
+    for B, H, mb, P in [(64, 128, 256, 74), (3, 32, 5, 3), (1, 16, 1, 1)]:
+        base = lib.mla_decode_workspace_bytes(B, H, P)
+        table = -(-base // 256) * 256
+        cache = -(-(table + 4 * B * mb) // 256) * 256
+        assert lib.mla_decode_fp8_workspace_bytes(B, H, mb, P) == cache + B * mb * 64 * 576 * 2
+    assert lib.mla_decode_fp8_workspace_bytes(64, 128, 0, 74) == 0        # no table
+    assert lib.mla_decode_fp8_workspace_bytes(64, 100, 4, 74) == 0        # bad H
+    assert lib.mla_decode_fp8_workspace_bytes(4096, 128, 8192, 74) == 0   # 2^25 blocks > 2^24
+
+
 @pytest.mark.parametrize("case", ["null_q", "bad_heads", "bad_batch", "fp8_missing_rope",
                                   "bf16_with_scale", "bad_scale", "misaligned"])
 def test_decode_rejects_invalid_arguments_on_host(case):

@@ -55,9 +55,32 @@ def test_sharp_softmax():
     check_full(w, 5, what="sharp")
 
 
-def test_fp8_cache_small():
+@pytest.mark.parametrize("route", ["tensor", "cuda-core"])
+def test_fp8_cache_small(route):
+    """The fp8 cache through the widened bf16 copy (workspace sized by
+    mla_decode_fp8_workspace_bytes) and through the CUDA-core decode (a
+    workspace of mla_decode_workspace_bytes, no room for the copy)."""
     w = inputs.make("fp8", B=3, H=32, L=[200, 64, 1], seed=24, q_std=2.0, extra_blocks=2)
-    check_full(w, 3, what="fp8")
+    d = binding.to_device(w)
+    ws = None if route == "tensor" else binding.alloc_workspace(w.B, w.H, 3)
+    out, lse, ws = binding.decode_device(d, w.softmax_scale, num_splits=3, workspace=ws)
+    assert binding.mla_get_device_error(ws) == 0
+    ro, rl = oracle.decode_workload(w)
+    assert_close(to_np(out).reshape(-1, 512), ro, f"fp8 {route} out")
+    assert_close(to_np(lse).reshape(-1), rl, f"fp8 {route} lse")
+
+
+def test_fp8_routes_agree_on_a_ragged_batch():
+    w = inputs.make("fp8", B=5, H=64, L=[1, 700, 65, 64, 2000], seed=33, q_std=3.0, extra_blocks=3)
+    d = binding.to_device(w)
+    o1, l1, ws1 = binding.decode_device(d, w.softmax_scale, num_splits=4)
+    o2, l2, ws2 = binding.decode_device(d, w.softmax_scale, num_splits=4,
+                                        workspace=binding.alloc_workspace(w.B, w.H, 4))
+    assert binding.mla_get_device_error(ws1) == 0 and binding.mla_get_device_error(ws2) == 0
+    ro, rl = oracle.decode_workload(w)
+    for o, l, what in ((o1, l1, "tensor"), (o2, l2, "cuda-core")):
+        assert_close(to_np(o).reshape(-1, 512), ro, f"fp8 {what} out")
+        assert_close(to_np(l).reshape(-1), rl, f"fp8 {what} lse")
 
 
 @pytest.mark.parametrize("cache", ["bf16", "fp8"])
@@ -112,11 +135,15 @@ def test_single_token_and_zero_query():
 
 # ---------------------------------------------------------------- device-side checks
 
-def test_bad_block_id_sets_error_bit():
-    w = inputs.make("v3", B=2, H=16, L=[100, 100], seed=30)
+@pytest.mark.parametrize("cache", ["bf16", "fp8"])
+def test_bad_block_id_sets_error_bit(cache):
+    w = inputs.make("v3", B=2, H=16, L=[100, 100], cache=cache, seed=30)
     w.block_table[1, 1] = w.num_blocks + 5
     out, lse, err = run(w)
     assert err & binding.DEVERR_BAD_BLOCK
+    # the rows of the other sequence are still right
+    ro, rl = oracle.decode_workload(w, rows=np.array([[0, h] for h in range(w.H)], np.int32))
+    assert_close(to_np(out)[0], ro, "good sequence next to a bad block")
 
 
 def test_seq_len_beyond_table_sets_error_bit():
