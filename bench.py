@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--json-out", default=None,
+                    help="also append the result line to this file (rank 0)")
     return ap.parse_args()
 
 
@@ -207,6 +209,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def nvtx_push(name: str):
+    """Named range for a profiler timeline (around whole regions, never per step)."""
+    try:
+        torch.cuda.nvtx.range_push(name)
+    except Exception:  # no NVTX library: the ranges are optional
+        pass
+
+
+def nvtx_pop():
+    try:
+        torch.cuda.nvtx.range_pop()
+    except Exception:
+        pass
+
+
 def step_bytes_flops(w):
     dec_b = layout.decode_algorithmic_bytes(w.total_tokens, w.B, w.H, w.cache_dtype,
                                             num_blocks_read=int(((w.seq_lens + 63) // 64).sum()))
@@ -247,9 +264,11 @@ def run_ours(args, world, rank, local):
                            lse, ws, k_rope=d["k_rope"], block_scale=d["block_scale"],
                            num_splits=args.num_splits, stream=stream)
 
+    nvtx_push("warm-up")
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize(dev)
+    nvtx_pop()
     if binding.mla_get_device_error(ws, stream) != 0:
         raise RuntimeError("device error during warm-up")
 
@@ -263,6 +282,7 @@ def run_ours(args, world, rank, local):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
+    nvtx_push("timed steps")
     t0.record(stream)
     for i in range(K):
         binding.mla_absorb_q(d["q_nope"], d["w_uk"], q_rope, q, stream=stream)
@@ -273,6 +293,7 @@ def run_ours(args, world, rank, local):
         ev_dec[i][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
+    nvtx_pop()
     if world > 1:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1)
@@ -299,6 +320,7 @@ def run_ours(args, world, rank, local):
     K2 = max(1, K // 2)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
+    nvtx_push("end-to-end steps")
     e0.record(stream)
     up.wait_event(e0)
     down.wait_event(e0)
@@ -327,6 +349,7 @@ def run_ours(args, world, rank, local):
         stream.wait_event(ev_out[k])
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    nvtx_pop()
     e2e_ms = e0.elapsed_time(e1) / K2
     clk = clocks.stop()
 
@@ -493,7 +516,16 @@ def run_reference(args, world, rank):
                              "sample": desc + " per step"},
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
+    emit(line, args.json_out)
+
+
+def emit(line: dict, path=None):
+    """Print the one JSON result line (and append it to ``path`` if given)."""
+    text = json.dumps(line)
+    print(text, flush=True)
+    if path:
+        with open(path, "a") as f:
+            f.write(text + "\n")
 
 
 def main():
@@ -508,7 +540,7 @@ def main():
             v, cores, desc, t = oracle_sample_rate(w, args.cpu_seconds)
             res["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores,
                                    "kind": "oracle", "sample": desc + f", {t:.1f} s"}
-        print(json.dumps(res), flush=True)
+        emit(res, args.json_out)
 
 
 if __name__ == "__main__":

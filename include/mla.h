@@ -148,7 +148,10 @@ size_t mla_decode_fp8_workspace_bytes(int B, int H, int max_blocks_per_seq, int 
  *              library keeps its error word zero except when it records an
  *              error.  One workspace must not be shared by calls that may run
  *              at the same time.
- * num_splits:  number of split-KV partitions (0 = automatic).  Results do not
+ * num_splits:  number of split-KV partitions (0 = automatic: the environment
+ *              variable MLA_SPLITS, read once per process, when it holds an
+ *              integer in 1..4096; else chosen from the device's SM count and
+ *              B, the same in mla_decode_workspace_bytes).  Results do not
  *              depend on the physical block placement; they may differ in the
  *              last bits between different num_splits.
  *

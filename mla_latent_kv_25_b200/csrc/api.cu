@@ -2,6 +2,8 @@
 // workspace layout, choice of the split-KV engine count, and the launches.
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <stdlib.h>
+
 #include <atomic>
 #include <mutex>
 
@@ -42,6 +44,24 @@ int device_max_clusters() {
   return cache[dev];
 }
 
+constexpr int kMaxSplits = 4096;
+
+// MLA_SPLITS=<1..4096> in the environment (read once) replaces the automatic
+// engine count; anything else leaves it automatic.
+int env_splits() {
+  static int value = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    value = 0;
+    const char* s = getenv("MLA_SPLITS");
+    if (s == nullptr || *s == '\0') return;
+    char* end = nullptr;
+    const long v = strtol(s, &end, 10);
+    if (end != nullptr && *end == '\0' && v >= 1 && v <= kMaxSplits) value = static_cast<int>(v);
+  });
+  return value;
+}
+
 // Engines of the split-KV partition.  By default one per co-resident cluster
 // of two SMs; but when the batch is at least three quarters of that and the
 // sequences are of similar length, one engine per sequence is faster: no
@@ -49,6 +69,7 @@ int device_max_clusters() {
 // single segment, which outweighs the idle clusters.
 int resolve_engines(int num_splits, int B) {
   if (num_splits > 0) return num_splits;
+  if (const int env = env_splits(); env > 0) return env;
   int sms = device_sms();
   if (sms < 2) return 0;
   int P = sms / 2;
@@ -94,7 +115,6 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
   return encode_bf16(map, base, 2, dims, strides, box);
 }
 
-constexpr int kMaxSplits = 4096;
 constexpr int kMaxBatch = 1 << 20;
 constexpr long long kDefaultSpin = 4000000000LL;  // ~2 s of SM clock
 std::atomic<long long> g_decode_wait_limit{kDefaultSpin};  // set by mla_set_wait_limit

@@ -4,6 +4,8 @@ before touching the device."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -50,6 +52,30 @@ def test_workspace_size_and_validation_without_device():
     assert lib.mla_decode_workspace_bytes(64, 256, 74) == 0     # H > 128
     assert lib.mla_decode_workspace_bytes(0, 128, 74) == 0
     assert lib.mla_decode_workspace_bytes(1, 128, -1) == 0
+
+
+def _workspace_in_child(env_value):
+    code = ("from mla_latent_kv_25_b200 import binding; "
+            "print(binding.load().mla_decode_workspace_bytes(64, 128, 0))")
+    env = dict(os.environ)
+    env.pop("MLA_SPLITS", None)
+    if env_value is not None:
+        env["MLA_SPLITS"] = env_value
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=120)
+    assert r.returncode == 0, r.stderr[-2000:]
+    return int(r.stdout.strip().splitlines()[-1])
+
+
+def test_env_split_count_replaces_the_automatic_one():
+    """MLA_SPLITS=<1..4096> sets the split count that num_splits = 0 means;
+    other values leave the automatic count."""
+    lib = binding.load()
+    auto = _workspace_in_child(None)
+    assert _workspace_in_child("5") == lib.mla_decode_workspace_bytes(64, 128, 5)
+    assert _workspace_in_child("4096") == lib.mla_decode_workspace_bytes(64, 128, 4096)
+    for bad in ("0", "-3", "4097", "abc", "7x", ""):
+        assert _workspace_in_child(bad) == auto, bad
 
 
 def test_fp8_workspace_adds_the_widened_copy():
