@@ -16,8 +16,9 @@
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers unless stated otherwise, owned by
- *     the caller.  The library allocates no memory and never synchronises the
- *     stream (except mla_get_device_error, which says so).
+ *     the caller.  No call allocates memory (mla_decode_noalloc's scratch is a
+ *     file-scope array that exists from load time), and no call synchronises
+ *     the stream except the three *_get_error calls, which say so.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     All work is enqueued on it in order.
  *   - Arguments are validated on the host before anything is launched; a
@@ -177,8 +178,8 @@ mla_status_t mla_decode(const void *q, mla_cache_dtype_t cache_dtype, const void
  * token: it attends to the first seq_lens[b] - (q_len - 1 - j) cached tokens
  * (the drafts' own rows are already in the cache; causal among the drafts).
  * q: bf16 [B, q_len, H, 576]; out: bf16 [B, q_len, H, 512]; lse: f32
- * [B, q_len, H]; bf16 cache only (the fp8 cache returns MLA_ERR_UNSUPPORTED
- * for q_len > 1).  q_len * H must be a multiple of 16 and at most 128.
+ * [B, q_len, H]; bf16 cache only.  q_len * H must be a multiple of 16 and at
+ * most 128.
  * workspace: mla_decode_workspace_bytes(B, q_len * H, num_splits) bytes.
  * Other arguments and error behaviour as mla_decode; a token that sees no
  * cached token gives out = 0 and lse = -inf.
@@ -206,7 +207,8 @@ mla_status_t mla_combine(const float *o_part, const float *lse_part, int B, int 
  * mla_get_device_error - wait for `stream`, read the MLA_DEVERR_* bits that
  * kernels using `workspace` recorded, and reset them to zero.  *err_bits
  * receives the bits.  Returns MLA_OK, or MLA_ERR_CUDA if the stream or copy
- * failed.  This is the only entry point that synchronises.
+ * failed.  It synchronises the stream (as do mla_absorb_get_error and
+ * mla_cache_get_error; no other call does).
  */
 mla_status_t mla_get_device_error(void *workspace, void *stream, uint32_t *err_bits);
 
