@@ -13,6 +13,8 @@
 // TMEM lanes (= 32 batch rows) and writes bf16 rows.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -274,15 +276,16 @@ absorb_o_sm100_kernel(const __grid_constant__ CUtensorMap omap, const __grid_con
 
 cudaError_t launch_absorb_o(const CUtensorMap& omap, const CUtensorMap& wmap, __nv_bfloat16* out,
                             int ldo, int B, int H, long long spin_limit, cudaStream_t stream) {
-  static bool attr_set[64] = {false};
+  // per device, set once (host threads may race to set it; setting it twice is harmless)
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(absorb_o_sm100_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(kOSmem));
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   dim3 grid(H, (B + 127) / 128);
   absorb_o_sm100_kernel<<<grid, kThreads, kOSmem, stream>>>(omap, wmap, out, ldo, B, H, spin_limit);
@@ -292,15 +295,16 @@ cudaError_t launch_absorb_o(const CUtensorMap& omap, const CUtensorMap& wmap, __
 cudaError_t launch_absorb_q(const CUtensorMap& qmap, const CUtensorMap& wmap,
                             const __nv_bfloat16* q_rope, __nv_bfloat16* q_out, int ldq, int B,
                             int H, long long spin_limit, cudaStream_t stream) {
-  static bool attr_set[64] = {false};
+  // per device, set once (host threads may race to set it; setting it twice is harmless)
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(absorb_sm100_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   dim3 grid(H, (B + 127) / 128);
   absorb_sm100_kernel<<<grid, kThreads, kSmem, stream>>>(qmap, wmap, q_rope, q_out, ldq, B, H,
