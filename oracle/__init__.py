@@ -28,6 +28,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "mla_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "_build", "liboracle.so")
+# a prebuilt oracle library to load instead (the mutation test points the pins
+# at deliberately broken copies this way); it is used as it is, never rebuilt
+_LIB_OVERRIDE = os.environ.get("MLA_ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
@@ -51,8 +54,11 @@ def lib():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            L = ctypes.CDLL(_LIB_PATH)
+            if _LIB_OVERRIDE:
+                L = ctypes.CDLL(_LIB_OVERRIDE)
+            else:
+                build()
+                L = ctypes.CDLL(_LIB_PATH)
             vp, i32p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)
             L.orc_decode_units.restype = ctypes.c_int
             L.orc_decode_units.argtypes = [ctypes.c_int, vp, ctypes.c_int, vp, vp, vp, vp, vp,
