@@ -1,9 +1,12 @@
 """The oracle's pins catch plausible mistakes: each mutant below plants one
-mistake in a copy of oracle/mla_oracle.c (a dropped term, a wrong bias, a
-wrong index, a missing normalisation), compiles it, and runs the pins of
-tests/test_oracle_pins.py against it in a child process, which must fail.
-The unmutated copy, built the same way, must pass.  Nothing under oracle/
-is modified; the child loads the copy through MLA_ORACLE_LIB.
+mistake in a copy of the oracle (a dropped term, a wrong bias, a wrong index,
+a missing normalisation, a wrong rounding rule), and the pins of
+tests/test_oracle_pins.py (and, for the Python parts, tests/
+test_cache_oracle_pins.py) run against it in a child process, which must
+fail; the unmutated copy, run the same way, must pass.  Nothing under
+oracle/ is modified: a mutant of mla_oracle.c is compiled on its own and
+loaded through MLA_ORACLE_LIB; a mutant of a Python part runs in a scratch
+copy of the files the pins need.
 
 A mutant's anchor text must occur exactly once in the oracle source: when
 the oracle is edited, this test names the anchor to update."""
@@ -35,6 +38,61 @@ MUTANTS = {
         "for (int c = 0; c < ORC_DC; ++c) acc += orc_bf16_to_f64(w[c]) * orc_bf16_to_f64(o[c]);",
         "for (int c = 0; c < ORC_DC - 1; ++c) acc += orc_bf16_to_f64(w[c]) * orc_bf16_to_f64(o[c]);"),
 }
+
+
+# mistakes planted in the oracle's Python parts (file under oracle/, anchor, replacement)
+PY_MUTANTS = {
+    "RoPE rotation with a wrong sign": (
+        "naive.py", "out[..., 1::2] = x0 * s + x1 * c", "out[..., 1::2] = x0 * s - x1 * c"),
+    "unabsorbed values formed with W_UK": (
+        "naive.py", "v = c_kv @ w_uv[h].T", "v = c_kv @ w_uk[h].T"),
+    "E4M3 ties rounded to the odd code": (
+        "cache.py", "score = np.where(cand, 1 + 2 * even[None, :] + same_sign, 0)",
+        "score = np.where(cand, 1 + 2 * (1 - even[None, :]) + same_sign, 0)"),
+    "appended row one slot late": (
+        "cache.py", "return blocks, (pos % BLOCK).astype(np.int64), rows",
+        "return blocks, ((pos + 1) % BLOCK).astype(np.int64), rows"),
+}
+
+# the files a child run of the pins needs, copied into a scratch tree
+_TREE = ["oracle/__init__.py", "oracle/naive.py", "oracle/cache.py", "oracle/mla_oracle.c",
+         "mla_latent_kv_25_b200/__init__.py", "mla_latent_kv_25_b200/inputs.py",
+         "mla_latent_kv_25_b200/layout.py", "tests/__init__.py", "tests/conftest.py", "tests/_util.py",
+         "tests/test_oracle_pins.py", "tests/test_cache_oracle_pins.py"]
+
+
+def _tree_with(where, rel, old, new):
+    import shutil
+    for f in _TREE + [os.path.join("tests", "golden", g) for g in os.listdir(os.path.join(ROOT, "tests", "golden"))]:
+        src = os.path.join(ROOT, f)
+        if not os.path.exists(src):
+            continue
+        dst = where / f
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        shutil.copyfile(src, dst)
+    target = where / "oracle" / rel
+    text = target.read_text()
+    assert text.count(old) == 1, f"anchor not unique in oracle/{rel}: {old}"
+    target.write_text(text.replace(old, new))
+    env = dict(os.environ)
+    env.pop("MLA_ORACLE_LIB", None)
+    return subprocess.run([sys.executable, "-m", "pytest", str(where / "tests" / "test_oracle_pins.py"),
+                           str(where / "tests" / "test_cache_oracle_pins.py"), "-x", "-q",
+                           "-p", "no:cacheprovider"], cwd=str(where), env=env,
+                          capture_output=True, text=True, timeout=900)
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_pins_catch_the_python_mutant(name, tmp_path):
+    rel, old, new = PY_MUTANTS[name]
+    r = _tree_with(tmp_path, rel, old, new)
+    assert "passed" in r.stdout or "failed" in r.stdout, r.stdout[-2000:] + r.stderr[-2000:]
+    assert r.returncode != 0, f"mutant '{name}' passed every pin"
+
+
+def test_scratch_tree_without_a_mutant_passes_the_pins(tmp_path):
+    r = _tree_with(tmp_path, "naive.py", "import numpy as np", "import numpy as np")
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
 
 
 def _build(src_text, where):
