@@ -297,7 +297,9 @@ def run_ours(args, world, rank, local):
     if world > 1:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1)
-    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
+    dec_list = [a.elapsed_time(b) for a, b in ev_dec]
+    dec_ms = float(np.mean(dec_list))
+    dec_med, dec_min = float(np.median(dec_list)), float(np.min(dec_list))
 
     # end to end through the public API with host buffers, as a serving loop
     # runs it: every step copies its new queries (q_nope, q_rope) host->device
@@ -423,6 +425,8 @@ def run_ours(args, world, rank, local):
         roof["kernel"] = ("mla_decode (fp8 widening + decode kernel + merge kernel)" if fp8
                           else "mla_decode (decode kernel + merge kernel)")
         roof["ms_per_launch"] = round(dec_ms, 5)
+        roof["ms_per_launch_median"] = round(dec_med, 5)
+        roof["ms_per_launch_min"] = round(dec_min, 5)
         roof["roofline_ms"] = round(max(t_hbm, t_tc) * 1e3, 5)
         roof["peak_source"] = f"{src} ({'MEASURED_PEAKS.json' if src == 'measured' else 'fallback'})"
         res = {
