@@ -9,7 +9,6 @@ the method, and there is no fallback when the library is missing.
 from __future__ import annotations
 
 import ctypes
-import os
 import threading
 
 import torch

@@ -1,7 +1,6 @@
 """Pins of the cache-writer oracle (oracle/cache.py) against the format
 definitions and library routines."""
 import numpy as np
-import pytest
 import torch
 
 from oracle import cache, naive
