@@ -35,6 +35,22 @@ def test_library_exports_every_declared_symbol():
         assert isinstance(getattr(lib, n), ctypes._CFuncPtr)
 
 
+def test_error_codes_agree_across_header_kernels_and_binding():
+    """The status enum and device error bits of include/mla.h, the kernels'
+    error constants (csrc/common.cuh) and the binding's constants agree."""
+    hdr = open(os.path.join(ROOT, "include", "mla.h")).read()
+    enum = {n: int(v) for n, v in re.findall(r"\b(MLA_(?:OK|ERR_[A-Z_]+))\s*=\s*(\d+)", hdr)}
+    assert {binding.STATUS[v]: v for v in binding.STATUS} == enum
+    bits = {n: int(v, 16) for n, v in re.findall(r"#define (MLA_DEVERR_[A-Z_]+)\s+0x([0-9a-fA-F]+)u", hdr)}
+    assert bits == {"MLA_DEVERR_BAD_BLOCK": binding.DEVERR_BAD_BLOCK,
+                    "MLA_DEVERR_SEQ_TOO_LONG": binding.DEVERR_SEQ_TOO_LONG,
+                    "MLA_DEVERR_TIMEOUT": binding.DEVERR_TIMEOUT}
+    common = open(os.path.join(ROOT, "mla_latent_kv_25_b200", "csrc", "common.cuh")).read()
+    kern = {n: int(v, 16) for n, v in re.findall(r"constexpr uint32_t (kErr[A-Za-z]+) = 0x([0-9a-fA-F]+)u;", common)}
+    assert kern == {"kErrBadBlock": bits["MLA_DEVERR_BAD_BLOCK"], "kErrSeqTooLong": bits["MLA_DEVERR_SEQ_TOO_LONG"],
+                    "kErrTimeout": bits["MLA_DEVERR_TIMEOUT"]}
+
+
 def test_status_strings():
     for code, name in binding.STATUS.items():
         assert binding.mla_status_string(code) == name
