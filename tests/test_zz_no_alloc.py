@@ -61,3 +61,21 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
         torch.cuda.synchronize()
         assert_close(to_np(out).reshape(-1, 512), to_np(ref_out).reshape(-1, 512), "noalloc out")
         assert_close(to_np(lse).reshape(-1), to_np(ref_lse).reshape(-1), "noalloc lse")
+
+
+@pytest.mark.gpu
+def test_noalloc_fp8_cache_matches_decode():
+    """An fp8 cache through the built-in scratch: small enough that its
+    widened copy fits there, so it takes the tensor-core route as mla_decode
+    does with an fp8-sized workspace."""
+    w = inputs.make("fp8", B=3, H=32, L=[200, 64, 1], seed=47, q_std=2.0, extra_blocks=2)
+    d = binding.to_device(w)
+    ref_out, ref_lse, ws = binding.decode_device(d, w.softmax_scale, num_splits=3)
+    assert binding.mla_get_device_error(ws) == 0
+    out = torch.full((w.B, w.H, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((w.B, w.H), float("nan"), dtype=torch.float32, device="cuda")
+    st = _noalloc_raw(d, w, out, lse, 3)
+    assert st == 0, binding.STATUS.get(st, st)
+    torch.cuda.synchronize()
+    assert_close(to_np(out).reshape(-1, 512), to_np(ref_out).reshape(-1, 512), "noalloc fp8 out")
+    assert_close(to_np(lse).reshape(-1), to_np(ref_lse).reshape(-1), "noalloc fp8 lse")
