@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--workload", default="v3", choices=list(inputs.CONFIGS))
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="skip the decode timings of the ragged, long and fp8 configurations")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--json-out", default=None,
@@ -233,6 +235,136 @@ def step_bytes_flops(w):
     return dec_b, abs_b, dec_f, abs_f
 
 
+def time_launches(fn, n: int, stream):
+    """Per-launch device times (ms) of ``n`` back-to-back calls of ``fn``,
+    each bracketed by CUDA events recorded on ``stream`` (the stream the
+    kernels are launched on)."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def roofline_block(dec_b: int, dec_f: int, ms_list, peaks: dict, src: str, kernel: str,
+                   traffic=None, launches: int = 0) -> dict:
+    """Roofline of one decode call: the slower of its algorithmic bytes at the
+    measured HBM copy bandwidth and its FLOPs at the measured dense bf16 peak
+    (burst: the call is timed on its own); achieved = algorithmic units over
+    the mean CUDA-event duration of the call."""
+    hbm = float(peaks["hbm_gbs"])
+    tens = float(peaks["bf16_tflops"])
+    ms = float(np.mean(ms_list))
+    t_hbm = dec_b / (hbm * 1e9)
+    t_tc = dec_f / (tens * 1e12)
+    if t_hbm >= t_tc:
+        achieved = dec_b / (ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4)}
+    else:
+        achieved = dec_f / (ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tens,
+                "unit": "TFLOP/s", "frac": round(achieved / tens, 4)}
+    roof.update({
+        "traffic": traffic, "algorithmic_bytes": int(dec_b), "flops": int(dec_f),
+        "kernel": kernel, "launches_timed": len(ms_list), "kernels_per_call": launches,
+        "ms_per_launch": round(ms, 5),
+        "ms_per_launch_median": round(float(np.median(ms_list)), 5),
+        "ms_per_launch_min": round(float(np.min(ms_list)), 5),
+        "roofline_ms": round(max(t_hbm, t_tc) * 1e3, 5),
+        "achieved_gbs": round(dec_b / (ms * 1e-3) / 1e9, 1),
+        "achieved_tflops": round(dec_f / (ms * 1e-3) / 1e12, 1),
+        "peak_source": f"{src} ({'MEASURED_PEAKS.json' if src == 'measured' else 'fallback'})",
+    })
+    return roof
+
+
+def decode_kernels_per_call(fp8: bool) -> int:
+    """Kernels one mla_decode call launches: the decode kernel and the merge
+    (an fp8 cache adds its widening kernel)."""
+    return 3 if fp8 else 2
+
+
+def fp8_through_writers(binding, name: str, dev, stream):
+    """The fp8 workload built the way a serving stack fills its cache: the
+    seeded rows (c_kv and the key before rotation) are appended through
+    mla_cache_append (RoPE in fp32, bf16 rows) and every block is converted
+    by mla_cache_quantize_fp8 (per-block scale, E4M3 codes).  Returns the
+    workload (its bf16 draws) and the device tensors of the fp8 cache."""
+    w = inputs.make(name, cache="bf16")
+    d = binding.to_device(w, dev)
+    raw = d["cache"]
+    nb = ((w.seq_lens.to(torch.int64) + 63) // 64)
+    tok_b = torch.repeat_interleave(torch.arange(w.B), w.seq_lens.to(torch.int64))
+    starts = torch.cumsum(w.seq_lens.to(torch.int64), 0) - w.seq_lens.to(torch.int64)
+    tok_p = torch.arange(int(w.seq_lens.sum())) - torch.repeat_interleave(starts, w.seq_lens.to(torch.int64))
+    phys = w.block_table[tok_b, tok_p // 64].to(torch.int64)
+    rows = raw[phys.to(dev), (tok_p % 64).to(dev)]                # [T, 576] draws
+    c_kv = rows[:, :512].contiguous()
+    k_r = rows[:, 512:].contiguous()
+    cache_bf16 = torch.zeros_like(raw)
+    binding.mla_cache_append(c_kv, k_r, tok_b.to(torch.int32).to(dev), tok_p.to(torch.int32).to(dev),
+                             d["block_table"], cache_bf16, stream=stream)
+    NB = int(raw.shape[0])
+    codes = torch.empty((NB, 64, 512), dtype=torch.uint8, device=dev)
+    k_rope = torch.empty((NB, 64, 64), dtype=torch.bfloat16, device=dev)
+    scale = torch.empty((NB,), dtype=torch.float32, device=dev)
+    binding.mla_cache_quantize_fp8(cache_bf16, torch.arange(NB, dtype=torch.int32, device=dev),
+                                   codes, k_rope, scale, stream=stream)
+    if binding.mla_cache_get_error(stream) != 0:
+        raise RuntimeError("device error in the cache writers")
+    del rows, c_kv, k_r, cache_bf16, raw
+    d["cache"], d["k_rope"], d["block_scale"] = codes, k_rope, scale
+    assert int(nb.sum()) <= NB
+    return w, d
+
+
+def extra_workload(binding, name: str, dev, stream, peaks, src, n_launch: int, num_splits: int):
+    """Decode-only timing of another configuration (absorbed queries as
+    drawn), with its own roofline block."""
+    if name == "fp8":
+        w, d = fp8_through_writers(binding, name, dev, stream)
+        fp8 = True
+        kind = "fp8"
+    else:
+        w = inputs.make(name)
+        d = binding.to_device(w, dev)
+        fp8 = False
+        kind = w.cache_dtype
+    B, H = w.B, w.H
+    out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    ws = binding.alloc_workspace(B, H, num_splits, device=dev,
+                                 fp8_max_blocks=int(w.block_table.shape[1]) if fp8 else None)
+
+    def call():
+        binding.mla_decode(d["q"], d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale, out,
+                           lse, ws, k_rope=d["k_rope"], block_scale=d["block_scale"],
+                           num_splits=num_splits, stream=stream)
+
+    for _ in range(5):
+        call()
+    ms = time_launches(call, n_launch, stream)
+    if binding.mla_get_device_error(ws, stream) != 0:
+        raise RuntimeError(f"device error in the {name} decode")
+    nblk = int(((w.seq_lens + 63) // 64).sum())
+    dec_b = layout.decode_algorithmic_bytes(w.total_tokens, B, H, kind, num_blocks_read=nblk)
+    dec_f = layout.decode_flops(w.total_tokens, H)
+    roof = roofline_block(dec_b, dec_f, ms, peaks, src,
+                          "mla_decode" + (" (fp8 cache)" if fp8 else ""),
+                          traffic=stored_traffic(name), launches=decode_kernels_per_call(fp8))
+    roof["description"] = inputs.DESCRIPTIONS[name] + (
+        "; cache built by mla_cache_append (RoPE in fp32) + mla_cache_quantize_fp8" if fp8 else "")
+    roof["tokens"] = w.total_tokens
+    del d, out, lse, ws
+    torch.cuda.empty_cache()
+    return roof
+
+
 def run_ours(args, world, rank, local):
     from mla_latent_kv_25_b200 import binding
 
@@ -251,21 +383,25 @@ def run_ours(args, world, rank, local):
     out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, H), dtype=torch.float32, device=dev)
     fp8 = w.cache_dtype != "bf16"
-    # an fp8 cache runs on the tensor cores through its widened bf16 copy,
-    # which the workspace holds: one more kernel per step
     ws = binding.alloc_workspace(B, H, args.num_splits, device=dev,
                                  fp8_max_blocks=int(w.block_table.shape[1]) if fp8 else None)
-    launches_per_step = 4 if fp8 else 3
+    launches_per_step = 1 + decode_kernels_per_call(fp8)
     dec_b, abs_b, dec_f, abs_f = step_bytes_flops(w)
+    peaks, src = load_peaks()
+
+    def decode(qq=None, oo=None, ll=None):
+        binding.mla_decode(q if qq is None else qq, d["cache"], d["block_table"], d["seq_lens"],
+                           w.softmax_scale, out if oo is None else oo, lse if ll is None else ll,
+                           ws, k_rope=d["k_rope"], block_scale=d["block_scale"],
+                           num_splits=args.num_splits, stream=stream)
 
     def step():
         binding.mla_absorb_q(d["q_nope"], d["w_uk"], q_rope, q, stream=stream)
-        binding.mla_decode(q, d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale, out,
-                           lse, ws, k_rope=d["k_rope"], block_scale=d["block_scale"],
-                           num_splits=args.num_splits, stream=stream)
+        decode()
 
+    W = max(3, args.warmup)
     nvtx_push("warm-up")
-    for _ in range(max(3, args.warmup)):
+    for _ in range(W):
         step()
     torch.cuda.synchronize(dev)
     nvtx_pop()
@@ -274,38 +410,37 @@ def run_ours(args, world, rank, local):
 
     clocks = ClockSampler(local)
     clocks.start()
-    # device-timed region: K steps, decode calls bracketed by events as well
+    # device-timed region: exactly K steps between a barrier + synchronize on
+    # each side
     K = args.steps
-    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     nvtx_push("timed steps")
     t0.record(stream)
-    for i in range(K):
-        binding.mla_absorb_q(d["q_nope"], d["w_uk"], q_rope, q, stream=stream)
-        ev_dec[i][0].record(stream)
-        binding.mla_decode(q, d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale, out,
-                           lse, ws, k_rope=d["k_rope"], block_scale=d["block_scale"],
-                           num_splits=args.num_splits, stream=stream)
-        ev_dec[i][1].record(stream)
+    for _ in range(K):
+        step()
     t1.record(stream)
     torch.cuda.synchronize(dev)
     nvtx_pop()
     if world > 1:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1)
-    dec_list = [a.elapsed_time(b) for a, b in ev_dec]
+
+    # the dominant call, timed on its own over many back-to-back launches
+    n_dec = max(200, K)
+    nvtx_push("decode launches")
+    dec_list = time_launches(decode, n_dec, stream)
+    nvtx_pop()
     dec_ms = float(np.mean(dec_list))
-    dec_med, dec_min = float(np.median(dec_list)), float(np.min(dec_list))
 
     # end to end through the public API with host buffers, as a serving loop
     # runs it: every step copies its new queries (q_nope, q_rope) host->device
     # and its out/lse device->host; inputs and outputs are double-buffered and
     # the copies run on their own streams, so step i+1's upload and step i's
-    # download overlap step i's compute.  All copies lie inside the timed region.
+    # download overlap step i's compute.  All copies lie inside the timed
+    # region; a few untimed steps of the same loop come first.
     h_qn = w.q_nope.pin_memory()
     h_qr = w.q[:, :, 512:].contiguous().pin_memory()
     h_out = [torch.empty((B, H, 512), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
@@ -316,59 +451,55 @@ def run_ours(args, world, rank, local):
     d_out = [out, torch.empty_like(out)]
     d_lse = [lse, torch.empty_like(lse)]
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer k uploaded
-    ev_done = [torch.cuda.Event() for _ in range(2)]   # step on buffer k computed
-    ev_out = [torch.cuda.Event() for _ in range(2)]    # results of buffer k downloaded
-    K2 = max(1, K // 2)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(dev)
+
+    def e2e_loop(n):
+        ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer k uploaded
+        ev_done = [torch.cuda.Event() for _ in range(2)]   # step on buffer k computed
+        ev_out = [torch.cuda.Event() for _ in range(2)]    # results of buffer k downloaded
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        up.wait_event(e0)
+        down.wait_event(e0)
+        for i in range(n):
+            k = i & 1
+            if i >= 2:
+                up.wait_event(ev_done[k])          # step i-2 has read input buffer k
+            with torch.cuda.stream(up):
+                d_qn[k].copy_(h_qn, non_blocking=True)
+                d_qr[k].copy_(h_qr, non_blocking=True)
+            ev_in[k].record(up)
+            stream.wait_event(ev_in[k])
+            if i >= 2:
+                stream.wait_event(ev_out[k])       # step i-2's results have left buffer k
+            binding.mla_absorb_q(d_qn[k], d["w_uk"], d_qr[k], d_q[k], stream=stream)
+            decode(d_q[k], d_out[k], d_lse[k])
+            ev_done[k].record(stream)
+            down.wait_event(ev_done[k])
+            with torch.cuda.stream(down):
+                h_out[k].copy_(d_out[k], non_blocking=True)
+                h_lse[k].copy_(d_lse[k], non_blocking=True)
+            ev_out[k].record(down)
+        for k in range(min(2, n)):
+            stream.wait_event(ev_out[k])
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n
+
+    e2e_loop(W)                        # untimed: first copies on fresh streams and buffers
+    K2 = max(200, K)
     nvtx_push("end-to-end steps")
-    e0.record(stream)
-    up.wait_event(e0)
-    down.wait_event(e0)
-    for i in range(K2):
-        k = i & 1
-        if i >= 2:
-            up.wait_event(ev_done[k])          # step i-2 has read input buffer k
-        with torch.cuda.stream(up):
-            d_qn[k].copy_(h_qn, non_blocking=True)
-            d_qr[k].copy_(h_qr, non_blocking=True)
-        ev_in[k].record(up)
-        stream.wait_event(ev_in[k])
-        if i >= 2:
-            stream.wait_event(ev_out[k])       # step i-2's results have left buffer k
-        binding.mla_absorb_q(d_qn[k], d["w_uk"], d_qr[k], d_q[k], stream=stream)
-        binding.mla_decode(d_q[k], d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale,
-                           d_out[k], d_lse[k], ws, k_rope=d["k_rope"], block_scale=d["block_scale"],
-                           num_splits=args.num_splits, stream=stream)
-        ev_done[k].record(stream)
-        down.wait_event(ev_done[k])
-        with torch.cuda.stream(down):
-            h_out[k].copy_(d_out[k], non_blocking=True)
-            h_lse[k].copy_(d_lse[k], non_blocking=True)
-        ev_out[k].record(down)
-    for k in range(min(2, K2)):
-        stream.wait_event(ev_out[k])
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    e2e_ms = e2e_loop(K2)
     nvtx_pop()
-    e2e_ms = e0.elapsed_time(e1) / K2
     clk = clocks.stop()
 
     # the step after the hot path, timed on its own (not part of the step):
     # output absorption out_h = W_UV[h] . o_latent on this step's output
     o_heads = torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev)
-    K3 = 200
     for _ in range(3):
         binding.mla_absorb_o(out, d["w_uv"], o_heads, stream=stream)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(dev)
-    a0.record(stream)
-    for _ in range(K3):
-        binding.mla_absorb_o(out, d["w_uv"], o_heads, stream=stream)
-    a1.record(stream)
-    torch.cuda.synchronize(dev)
-    absorb_o_ms = a0.elapsed_time(a1) / K3
+    absorb_o_ms = float(np.mean(time_launches(
+        lambda: binding.mla_absorb_o(out, d["w_uv"], o_heads, stream=stream), 200, stream)))
     if binding.mla_absorb_get_error(stream) != 0:
         raise RuntimeError("device error in the output absorption")
 
@@ -380,62 +511,49 @@ def run_ours(args, world, rank, local):
         out2 = torch.empty((B, 2, H // 2, 512), dtype=torch.bfloat16, device=dev)
         lse2 = torch.empty((B, 2, H // 2), dtype=torch.float32, device=dev)
         ws2 = binding.alloc_workspace(B, H, args.num_splits, device=dev)
+
+        def mcall():
+            binding.mla_decode_multi(q2, d["cache"], d["block_table"], d["seq_lens"],
+                                     w.softmax_scale, out2, lse2, ws2, num_splits=args.num_splits,
+                                     stream=stream)
         for _ in range(3):
-            binding.mla_decode_multi(q2, d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale,
-                                     out2, lse2, ws2, num_splits=args.num_splits, stream=stream)
-        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize(dev)
-        K4 = 50
-        m0.record(stream)
-        for _ in range(K4):
-            binding.mla_decode_multi(q2, d["cache"], d["block_table"], d["seq_lens"], w.softmax_scale,
-                                     out2, lse2, ws2, num_splits=args.num_splits, stream=stream)
-        m1.record(stream)
-        torch.cuda.synchronize(dev)
+            mcall()
+        m_ms = float(np.mean(time_launches(mcall, 100, stream)))
         if binding.mla_get_device_error(ws2, stream) != 0:
             raise RuntimeError("device error in the multi-token decode")
-        multi = {"q_len": 2, "heads": H // 2, "ms_per_launch": round(m0.elapsed_time(m1) / K4, 5)}
+        multi = {"q_len": 2, "heads_per_token": H // 2, "rows_per_sequence": H,
+                 "note": "the same query rows regrouped as 2 draft tokens x H/2 heads",
+                 "ms_per_launch": round(m_ms, 5)}
     if binding.mla_get_device_error(ws, stream) != 0:
         raise RuntimeError("device error during timing")
 
     step_ms = ms / K
     step_ms, dec_ms, e2e_ms = max_over_ranks([step_ms, dec_ms, e2e_ms], dev)
 
+    extras = {}
+    if world == 1 and args.workload == "v3" and not args.no_extra_workloads:
+        del ws
+        for name in ("ragged", "long", "fp8"):
+            extras[name] = extra_workload(binding, name, dev, stream, peaks, src, 100,
+                                          args.num_splits)
+
     res = None
     if rank == 0:
-        peaks, src = load_peaks()
-        hbm = float(peaks["hbm_gbs"])
-        tens = float(peaks["bf16_tflops"])
         step_bytes = dec_b + abs_b
         value = job_rate(step_bytes, world, step_ms)
-        achieved = dec_b / (dec_ms * 1e-3) / 1e9
-        dec_tflops = dec_f / (dec_ms * 1e-3) / 1e12
-        t_hbm = dec_b / (hbm * 1e9)
-        t_tc = dec_f / (tens * 1e12)
-        bound = "hbm" if t_hbm >= t_tc else "tensor"
-        traffic = stored_traffic(args.workload)
-        if bound == "hbm":
-            roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(achieved / hbm, 4)}
-        else:
-            roof = {"bound": "tensor", "achieved": round(dec_tflops, 1), "peak": tens,
-                    "unit": "TFLOP/s", "frac": round(dec_tflops / tens, 4)}
-        roof["traffic"] = traffic
-        roof["algorithmic_bytes"] = dec_b
-        roof["kernel"] = ("mla_decode (fp8 widening + decode kernel + merge kernel)" if fp8
-                          else "mla_decode (decode kernel + merge kernel)")
-        roof["ms_per_launch"] = round(dec_ms, 5)
-        roof["ms_per_launch_median"] = round(dec_med, 5)
-        roof["ms_per_launch_min"] = round(dec_min, 5)
-        roof["roofline_ms"] = round(max(t_hbm, t_tc) * 1e3, 5)
-        roof["peak_source"] = f"{src} ({'MEASURED_PEAKS.json' if src == 'measured' else 'fallback'})"
+        roof = roofline_block(dec_b, dec_f, dec_list, peaks, src,
+                              "mla_decode" + (" (fp8 cache)" if fp8 else ""),
+                              traffic=stored_traffic(args.workload),
+                              launches=decode_kernels_per_call(fp8))
+        if world > 1:
+            roof["ms_per_launch_max_over_ranks"] = round(dec_ms, 5)
         res = {
             "metric": METRIC,
             "value": round(value, 1),
             "unit": "GB/s",
             "n_gpus": world,
             "steps": K,
-            "warmup": max(3, args.warmup),
+            "warmup": W,
             "ms_per_step": round(step_ms, 5),
             "higher_is_better": True,
             "scaling": "weak",
@@ -449,18 +567,19 @@ def run_ours(args, world, rank, local):
                        "l2": "inputs larger than L2 (cache %.0f MB > 126 MB); no flush"
                              % (w.cache.numel() * w.cache.element_size() / 1e6)},
             "tflops": round((dec_f + abs_f) * world / (step_ms * 1e-3) / 1e12, 2),
-            "decode_tflops": round(dec_tflops, 2),
+            "decode_tflops": round(dec_f / (dec_ms * 1e-3) / 1e12, 2),
             "roofline": roof,
             "e2e": {"value": round(job_rate(step_bytes, world, e2e_ms), 1), "unit": "GB/s",
-                    "ms_per_step": round(e2e_ms, 5),
+                    "ms_per_step": round(e2e_ms, 5), "steps": K2,
                     "h2d_bytes_per_step": int(h_qn.numel() * 2 + h_qr.numel() * 2),
                     "d2h_bytes_per_step": int(h_out[0].numel() * 2 + h_lse[0].numel() * 4),
                     "pipelined": "double-buffered; copies on their own streams overlap compute"},
             "gpu_launches": launches_per_step * K,
-            "absorb_o": absorb_o_line(B, H, absorb_o_ms, hbm),
+            "absorb_o": absorb_o_line(B, H, absorb_o_ms, float(peaks["hbm_gbs"])),
             "multi_token": None if multi is None else dict(
                 multi, algorithmic_bytes=dec_b,
-                frac=round(dec_b / (multi["ms_per_launch"] * 1e-3) / 1e9 / hbm, 4)),
+                frac=round(dec_b / (multi["ms_per_launch"] * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4)),
+            "workloads": extras or None,
             "clocks": clk,
         }
     if world > 1:
@@ -478,7 +597,8 @@ def oracle_sample_rate(w, seconds: float, n_seq_max=None):
     rows = 0
     t_total = 0.0
     b = 0
-    while b < w.B and t_total < seconds and (n_seq_max is None or b < n_seq_max):
+    # at least one whole sequence, whatever the time budget
+    while b < w.B and (b == 0 or t_total < seconds) and (n_seq_max is None or b < n_seq_max):
         units = np.stack([np.full(w.H, b), np.arange(w.H), np.zeros(w.H), -np.ones(w.H)], 1)
         t = time.perf_counter()
         oracle.decode_units(q=w.q, cache=w.cache, block_table=w.block_table, seq_lens=w.seq_lens,

@@ -296,6 +296,13 @@ long long mla_set_wait_limit(long long cycles);
 /* mla_status_string - a static, human-readable name for a status code. */
 const char *mla_status_string(mla_status_t status);
 
+/*
+ * mla_last_error_string - a static description of the CUDA failure behind the
+ * last MLA_ERR_CUDA that a call made on this host thread returned ("no error"
+ * before any).  The pointer stays valid until the library is unloaded.
+ */
+const char *mla_last_error_string(void);
+
 /* mla_num_sms - streaming multiprocessors of the current device (0 on error). */
 int mla_num_sms(void);
 

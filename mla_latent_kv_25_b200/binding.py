@@ -32,12 +32,13 @@ EXPORTS = ("mla_absorb_q", "mla_absorb_o", "mla_absorb_get_error", "mla_cache_ap
            "mla_cache_quantize_fp8", "mla_cache_get_error", "mla_set_wait_limit", "mla_decode_multi",
            "mla_decode_workspace_bytes", "mla_decode_fp8_workspace_bytes", "mla_decode",
            "mla_combine", "mla_get_device_error", "mla_status_string", "mla_num_sms",
-           "mla_decode_noalloc")
+           "mla_decode_noalloc", "mla_last_error_string")
 
 
 class MLAError(RuntimeError):
-    def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        msg = f"{fn} returned {STATUS.get(status, status)}"
+        super().__init__(msg + (f" ({detail})" if detail else ""))
         self.status = status
 
 
@@ -88,6 +89,8 @@ def load():
         L.mla_status_string.argtypes = [i32]
         L.mla_num_sms.restype = i32
         L.mla_num_sms.argtypes = []
+        L.mla_last_error_string.restype = ctypes.c_char_p
+        L.mla_last_error_string.argtypes = []
         L.mla_decode_noalloc.restype = i32
         L.mla_decode_noalloc.argtypes = [vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                          ctypes.c_float, vp, vp, i32, vp]
@@ -107,7 +110,8 @@ def _stream(stream):
 
 def _check(fn, status):
     if status != MLA_OK:
-        raise MLAError(fn, status)
+        detail = load().mla_last_error_string().decode() if status == 4 else ""
+        raise MLAError(fn, status, detail)
 
 
 def _need(t, name, dtype, shape=None):

@@ -17,6 +17,22 @@ using namespace mla;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Text of the last CUDA failure a call on this host thread returned as
+// MLA_ERR_CUDA (mla_last_error_string).
+thread_local const char* g_last_error = "no error";
+
+mla_status_t cuda_fail(cudaError_t e) {
+  g_last_error = cudaGetErrorString(e);
+  return MLA_ERR_CUDA;
+}
+
+mla_status_t fail_with(const char* what) {
+  g_last_error = what;
+  return MLA_ERR_CUDA;
+}
+
+mla_status_t status_of(cudaError_t e) { return e == cudaSuccess ? MLA_OK : cuda_fail(e); }
+
 int device_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -191,13 +207,14 @@ mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, const void* q_ro
   const cuuint64_t qdims[3] = {cuuint64_t(kNope), cuuint64_t(H), cuuint64_t(B)};
   const cuuint64_t qstr[2] = {cuuint64_t(kNope) * 2, cuuint64_t(H) * kNope * 2};
   const cuuint32_t qbox[3] = {64, 1, 128};
-  if (!encode_bf16(&qmap, q_nope, 3, qdims, qstr, qbox)) return MLA_ERR_CUDA;
+  if (!encode_bf16(&qmap, q_nope, 3, qdims, qstr, qbox)) return fail_with("tensor map encoding failed");
   // W_UK [H, 128, 512] as rows (h, d) x columns c
-  if (!encode_bf16_map(&wmap, w_uk, uint64_t(H) * kNope, kDc, kDc * 2)) return MLA_ERR_CUDA;
+  if (!encode_bf16_map(&wmap, w_uk, uint64_t(H) * kNope, kDc, kDc * 2))
+    return fail_with("tensor map encoding failed");
   cudaError_t e = launch_absorb_q(qmap, wmap, static_cast<const __nv_bfloat16*>(q_rope),
                                   static_cast<__nv_bfloat16*>(q_out), ldq, B, H, kDefaultSpin,
                                   static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return status_of(e);
 }
 
 mla_status_t mla_absorb_o(const void* o_latent, const void* w_uv, void* out, int ldo, int B, int H,
@@ -211,15 +228,15 @@ mla_status_t mla_absorb_o(const void* o_latent, const void* w_uv, void* out, int
   const cuuint64_t odims[3] = {cuuint64_t(kDc), cuuint64_t(H), cuuint64_t(B)};
   const cuuint64_t ostr[2] = {cuuint64_t(kDc) * 2, cuuint64_t(H) * kDc * 2};
   const cuuint32_t obox[3] = {64, 1, 128};
-  if (!encode_bf16(&omap, o_latent, 3, odims, ostr, obox)) return MLA_ERR_CUDA;
+  if (!encode_bf16(&omap, o_latent, 3, odims, ostr, obox)) return fail_with("tensor map encoding failed");
   // W_UV [H, 128, 512] as rows (h, d) x columns c, one box = the 128 rows of a head
   const cuuint64_t wdims[2] = {cuuint64_t(kDc), cuuint64_t(H) * kNope};
   const cuuint64_t wstr[1] = {cuuint64_t(kDc) * 2};
   const cuuint32_t wbox[2] = {64, 128};
-  if (!encode_bf16(&wmap, w_uv, 2, wdims, wstr, wbox)) return MLA_ERR_CUDA;
+  if (!encode_bf16(&wmap, w_uv, 2, wdims, wstr, wbox)) return fail_with("tensor map encoding failed");
   cudaError_t e = launch_absorb_o(omap, wmap, static_cast<__nv_bfloat16*>(out), ldo, B, H,
                                   kDefaultSpin, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return status_of(e);
 }
 
 mla_status_t mla_cache_append(const void* c_kv, const void* k_r, const int32_t* seq_idx,
@@ -237,7 +254,7 @@ mla_status_t mla_cache_append(const void* c_kv, const void* k_r, const int32_t* 
                                       static_cast<const __nv_bfloat16*>(k_r), seq_idx, pos, T,
                                       block_table, B, max_blocks_per_seq, num_blocks,
                                       static_cast<__nv_bfloat16*>(cache), static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return status_of(e);
 }
 
 mla_status_t mla_cache_quantize_fp8(const void* cache_bf16, const int32_t* blocks, int n,
@@ -253,13 +270,14 @@ mla_status_t mla_cache_quantize_fp8(const void* cache_bf16, const int32_t* block
                                             num_blocks, static_cast<uint8_t*>(codes),
                                             static_cast<__nv_bfloat16*>(k_rope), block_scale,
                                             static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return status_of(e);
 }
 
 mla_status_t mla_cache_get_error(void* stream, uint32_t* err_bits) {
   if (!err_bits) return MLA_ERR_INVALID_ARG;
   uint32_t v = 0;
-  if (cache_take_error(&v, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaError_t e = cache_take_error(&v, static_cast<cudaStream_t>(stream)); e != cudaSuccess)
+    return cuda_fail(e);
   *err_bits = v;
   return MLA_OK;
 }
@@ -267,7 +285,8 @@ mla_status_t mla_cache_get_error(void* stream, uint32_t* err_bits) {
 mla_status_t mla_absorb_get_error(void* stream, uint32_t* err_bits) {
   if (!err_bits) return MLA_ERR_INVALID_ARG;
   uint32_t v = 0;
-  if (absorb_take_error(&v, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaError_t e = absorb_take_error(&v, static_cast<cudaStream_t>(stream)); e != cudaSuccess)
+    return cuda_fail(e);
   *err_bits = v;
   return MLA_OK;
 }
@@ -304,7 +323,7 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
       (block_scale && (reinterpret_cast<uintptr_t>(block_scale) & 3u) != 0))
     return MLA_ERR_INVALID_ARG;
   const int P = resolve_engines(num_splits, B);
-  if (P < 1) return MLA_ERR_CUDA;
+  if (P < 1) return fail_with("no streaming multiprocessor count for the current device");
   const WsLayout ws = ws_layout(B, rows, P);
   if (workspace_bytes < ws.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
 
@@ -345,7 +364,7 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
     e = launch_fp8_widen(static_cast<const uint8_t*>(cache), p.k_rope, block_scale, block_table,
                          seq_lens, B, max_blocks_per_seq, num_blocks, wide_table, wide_cache, p.err,
                          device_sms(), st);
-    if (e != cudaSuccess) return MLA_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e);
     p.cache = wide_cache;
     p.k_rope = nullptr;
     p.block_scale = nullptr;
@@ -355,15 +374,15 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
   if (!fp8 || widen) {
     CUtensorMap tmap;
     if (!encode_bf16_map(&tmap, p.cache, uint64_t(p.num_blocks) * kBlock, kRow, kRow * 2))
-      return MLA_ERR_CUDA;
+      return fail_with("tensor map encoding failed");
     e = launch_decode_sm100(p, tmap, st);
   } else {
     e = launch_decode_simt(p, fp8, st);
   }
-  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   e = launch_merge_pieces(seq_lens, B, max_blocks_per_seq, rows, p.seq_info, p.lse_part, p.o_part,
                           p.out, p.lse, p.err, st);
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return status_of(e);
 }
 
 }  // namespace
@@ -399,22 +418,24 @@ mla_status_t mla_combine(const float* o_part, const float* lse_part, int B, int 
     return MLA_ERR_INVALID_ARG;
   cudaError_t e = launch_combine(o_part, lse_part, B, H, S, static_cast<__nv_bfloat16*>(out), lse,
                                  static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return status_of(e);
 }
 
 mla_status_t mla_get_device_error(void* workspace, void* stream, uint32_t* err_bits) {
   if (!workspace || !err_bits) return MLA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t v = 0;
-  if (cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return MLA_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, st); e != cudaSuccess)
+    return cuda_fail(e);
+  if (cudaError_t e = cudaStreamSynchronize(st); e != cudaSuccess) return cuda_fail(e);
   *err_bits = v;
   if (v != 0) {
-    if (cudaMemsetAsync(workspace, 0, sizeof v, st) != cudaSuccess) return MLA_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof v, st); e != cudaSuccess) return cuda_fail(e);
+    if (cudaError_t e = cudaStreamSynchronize(st); e != cudaSuccess) return cuda_fail(e);
   }
   return MLA_OK;
 }
+
+const char* mla_last_error_string(void) { return g_last_error; }
 
 }  // extern "C"

@@ -21,7 +21,8 @@ constexpr uint32_t kErrTimeout = 0x4u;
 
 // ---------------------------------------------------------------------------
 // Workspace layout (all offsets 256-byte aligned):
-//   [0, 256)            header: uint32 error bits at offset 0
+//   [0, 256)            header: uint32 error bits at offset 0; at offsets 4 and 8
+//                       where the first timed-out wait gave up (diagnosis)
 //   seq_info  int4 [B]  per sequence: (first engine, last engine, slot of the
 //                       first engine's piece, kind) written by the decode
 //                       kernel, read by the merge kernel

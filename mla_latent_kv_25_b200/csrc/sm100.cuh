@@ -90,6 +90,8 @@ struct WaitCtx {
   long long limit;
   uint32_t* err;
   volatile int* abort;
+  uint32_t* where = nullptr;  // if set: [0] shared address of the first barrier that
+                              // timed out, [1] (block << 8) | warp that gave up
 };
 
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
@@ -125,9 +127,10 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // decode pipeline's hand-offs costs more than the issue slots polling takes.
 // Arguments by value: a reference would force the caller's context into
 // local memory, and every asm statement with a "memory" clobber (all the
-// barrier, TMA and MMA wrappers here) would then reload it.
-static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, long long limit,
-                                                    uint32_t* err, volatile int* abort) {
+// barrier, TMA and MMA wrappers here) would then reload it.  Inlined: a call
+// out of a region that runs under setmaxnreg cannot be register-allocated.
+static __device__ __forceinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, long long limit,
+                                                    uint32_t* err, volatile int* abort, uint32_t* where) {
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_test_wait(bar, parity)) return true;
@@ -135,6 +138,8 @@ static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parit
       if (*abort) return false;
       if (clock64() - t0 > limit) {
         atomicOr(err, kErrTimeout);
+        if (where != nullptr && atomicCAS(where, 0u, bar | 0x80000000u) == 0u)
+          where[1] = (blockIdx.x << 8) | (threadIdx.x >> 5);
         *abort = 1;
         return false;
       }
@@ -142,12 +147,10 @@ static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parit
   }
 }
 
-// The first probe is inlined; the polling loop is one out-of-line copy shared
-// by every wait site, which keeps the kernel's hot code small (each role's
-// warps run different code).
+// The first probe is tried before the polling loop.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_test_wait(bar, parity)) return true;
-  return wait_phase_slow(bar, parity, w.limit, w.err, w.abort);
+  return wait_phase_slow(bar, parity, w.limit, w.err, w.abort, w.where);
 }
 
 // Whole-warp wait: every lane waits (each takes its own acquire); the warp
@@ -238,6 +241,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_cluster_relaxed(uint32_t b
                    bar_cluster),
                "r"(bytes)
                : "memory");
+}
+
+// Register reallocation between warpgroups (all four warps of a warpgroup
+// execute it).  The sum over warpgroups must stay within the registers the
+// block was launched with (threads x registers per thread at launch).
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // 2^x on the special-function unit (flush-to-zero for tiny results).

@@ -76,7 +76,7 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero(tmp_path):
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
-           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "5",
            "--cpu-seconds", "0.3", "--workload", "tiny"]
     env = dict(os.environ, TMPDIR=str(tmp_path))  # torchrun's scratch files go to pytest's tmp dir
     r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
