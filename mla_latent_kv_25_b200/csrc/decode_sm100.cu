@@ -1,39 +1,44 @@
 // Absorbed MLA decode on sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
 // One split-KV engine = a cluster of two CTAs on two SMs, split by pipeline
-// role because the fp32 output accumulator of 128 heads x 512 latent columns
+// role, because the fp32 output accumulator of 128 heads x 512 latent columns
 // fills all 512 TMEM columns of one SM:
 //
-//   score CTA (rank 0)                           value CTA (rank 1)
-//   ------------------                           ------------------
-//   w0  TMA: cache rows of three 64-token         w0  TMA: latent part of each block,
-//       blocks per pass, one 64-column chunk          half a block (4 chunks) at a time
-//       at a time into a ring of [192 x 64] slots     into a ring of [64 x 256] slots
-//   w1  MMA: S = Q K^T for 192 tokens at once     w1  MMA: O += P V (A = P, B = V read
-//       (N = 192); Q columns 0..255 in TMEM,          MN-major), N = 256 per instruction
-//       columns 256..575 in shared memory         w2  zero V rows past seq_len
-//   w4-7 softmax, thread h = head h: online       w4-7 thread h = head h: rescale O rows
-//       softmax in fp32 per 64-token block;           when the running max grew; final
-//       P (bf16) and the rescale factors are         O / l and lse, or an fp32 piece of
-//       staged locally                                a cut sequence
-//   w2-3 senders: staged records -> value CTA
-//       with st.async (overlapping the softmax)
+//   score CTA (rank 0)                            value CTA (rank 1)
+//   ------------------                            ------------------
+//   w0    TMA: cache rows of a pass of four        w0    TMA: latent part of each block,
+//         64-token blocks, two 64-column chunks          half a block (4 chunks) per slot
+//         (64 KB) per ring slot                    w1    MMA: O += P V (A = P, B = V read
+//   w1    MMA: S = Q K^T for 256 tokens at once          MN-major), N = 256 per instruction
+//         (N = 256); Q columns 0..511 in TMEM      w2    zero V rows past seq_len
+//         (TS), the RoPE columns in shared memory  w4-11 thread = (head, latent half): O
+//   w4-11 softmax, thread = (head, half pass):            rescale when a max moved; final
+//         reads its 128 S columns at once (so the        O / l and lse, or an fp32 piece
+//         next pass's QK can start), online              of a cut sequence
+//         softmax in fp32, and sends P (bf16) and
+//         the per-head factors straight into the
+//         value CTA's shared memory (st.async)
 //
-// Why N = 192: inside this pipeline an MMA instruction costs roughly 100+
-// cycles to issue whatever its N, so 128-token passes ran the QK at half the
-// tensor pipe's rate; 192-token passes cut the instructions per block from 18
-// to 12.  Two 192-column S buffers leave TMEM room for only half of Q; the
-// rest of Q is an SS operand.
+// Why this shape (measured on B200): a single-CTA tcgen05.mma costs about
+// 120-135 cycles to issue whatever its N up to 192, so only N = 256 runs the
+// tensor pipe near its rate (the QK at ~141 cycles per 128-cycle instruction
+// with A in TMEM, the PV at ~129); an mbarrier probe between MMAs stalls the
+// issue stream unless it is issued ahead of the MMAs it guards, so every MMA
+// loop polls the next stage's barrier before issuing the current stage; the
+// SM-to-SM hand-off peaks at ~21 bytes per clock, enough for one 16 KB P tile
+// per block when 256 threads issue the stores.
+//
 // Heads are the M = 128 dimension of both contractions (padded with zero query
-// rows for H < 128).  The running max only moves when a block's max exceeds
-// it by more than 2^8 (log2 domain), so O is rarely rescaled.  Every wait is
-// bounded (WaitCtx); a timeout records an error bit and the CTA leaves its
-// loops, releases TMEM and exits.
+// rows for H < 128).  The running max of a head moves only when a pass's max
+// exceeds it by more than 2^8 (log2 domain), so O is rarely rescaled; both
+// softmax threads of a head take that decision on the same pass max.  Every
+// wait is bounded (WaitCtx); a timeout records an error bit and the CTA leaves
+// its loops, releases TMEM and exits.
 //
 // Barrier discipline: a parity wait can only tell the current phase from the
 // one before it, so every barrier here is either observed by its waiters at
 // every phase, in order, or used as a strict two-party handshake (q_ready /
-// q_free, pv_prev / corr_done, o_ready / o_free).
+// q_free, s_full / s_empty, epi_req / corr_done or o_free).
 #include <cuda.h>
 #include <math.h>
 
@@ -47,42 +52,45 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
-constexpr int kPassBlocks = 3;  // score CTA: blocks per QK pass, so N = 192 per MMA
-constexpr int kPassTok = kPassBlocks * 64;
-constexpr int kKSlots = 3;      // score CTA: ring of [192 tokens x 64 cols] slots, one column chunk each
-constexpr int kVSlots = 5;   // value CTA: ring of [64 tokens x 256 cols] half-block slots
-constexpr int kNP = 3;       // P records in flight
-constexpr int kNS = 2;       // S accumulators (128 columns each) in TMEM
+constexpr int kThreads = 384;                   // warpgroup 0: TMA, MMA; warpgroups 1-2: compute
+constexpr int kPassBlocks = 4;                  // score CTA: blocks per QK pass (N = 256)
+constexpr int kPassTok = kPassBlocks * kBlock;
+constexpr int kKSlots = 3;                      // score CTA: ring of two-chunk slots
+constexpr int kFills = 5;                       // slot fills per pass: chunks {0,1} {2,3} {4,5} {6,7} {8}
+constexpr int kVSlots = 4;                      // value CTA: ring of [64 x 256] half-block slots
+constexpr int kNP = 4;                          // P records in flight (value CTA)
 
-constexpr uint32_t kChunk = 64 * 128;          // one [64 rows x 64 bf16] swizzled chunk
-constexpr uint32_t kKSlot = kPassBlocks * kChunk;  // one column chunk of a pass: [192 rows x 64 bf16]
+constexpr uint32_t kChunk = 64 * 128;           // [64 rows x 64 bf16] swizzled (one block, one chunk)
+constexpr uint32_t kPassChunk = kPassBlocks * kChunk;  // one column chunk of a pass [256 x 64]
+constexpr uint32_t kKSlot = 2 * kPassChunk;     // two column chunks of a pass
 constexpr uint32_t kVSlot = 4 * kChunk;         // [64 rows x 256 bf16]
-constexpr uint32_t kPBytes = 128 * 64 * 2;     // P [128 heads x 64 tokens] bf16
-constexpr uint32_t kQTile = 128 * 64 * 2;      // one 64-column chunk of Q [128 heads x 64] bf16
-constexpr int kQTmemChunks = 4;                 // Q columns 0..255 live in TMEM (TS operand)
-constexpr int kQSmemTiles = 9 - kQTmemChunks;   // columns 256..575 in shared memory (SS operand)
-constexpr uint32_t kMetaWarp = 400;            // per warp: alpha[32] m[32] l[32] flag + pad
-constexpr uint32_t kMetaBytes = 4 * kMetaWarp;
-constexpr float kRescaleThreshold = 8.0f;      // log2 units
+constexpr uint32_t kPBytes = 128 * 64 * 2;      // P [128 heads x 64 tokens] bf16
+constexpr uint32_t kMetaBytes = 128 * 16;       // per head: alpha, m, l, unused
+constexpr uint32_t kFlagBytes = 64;             // per quadrant: rescale flag
+constexpr uint32_t kRecBytes = 19 * 1024;       // one record (P, meta, flags), 1 KB aligned
+constexpr uint32_t kQTile = 128 * 64 * 2;       // [128 heads x 64] bf16 (the RoPE columns of Q)
+constexpr int kQTmemChunks = 8;                 // Q columns 0..511 in TMEM (TS operand)
+constexpr float kRescaleThreshold = 8.0f;       // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
+static_assert(kPBytes + kMetaBytes + kFlagBytes <= kRecBytes, "record layout");
 
-// TMEM columns of the score CTA: Q columns 0..255 (bf16 pairs: 128 columns),
-// then two S buffers of kPassTok fp32 columns each.
-constexpr uint32_t kQCol = 0;
-constexpr uint32_t kSCol = kQTmemChunks * 32;
-static_assert(kSCol + 2 * kPassTok <= 512, "TMEM columns");
+// TMEM columns of the score CTA: S (fp32, one column per token of the pass),
+// then Q columns 0..511 as packed bf16 pairs (32 columns per 64-wide chunk).
+constexpr uint32_t kSCol = 0;
+constexpr uint32_t kQCol = kPassTok;
+static_assert(kQCol + kQTmemChunks * 32 <= 512, "TMEM columns");
 constexpr uint32_t kTmemCols = 512;
 
 struct Barriers {
   uint64_t k_full[kKSlots], k_empty[kKSlots];
-  uint64_t s_full[kNS], s_empty[kNS];
+  uint64_t s_full, s_empty;
   uint64_t q_ready, q_free;
-  uint64_t p_empty[kNP];
-  uint64_t stage_full[kNP], stage_empty[kNP];
+  uint64_t xchg[4];                 // softmax: the two threads of a head swap max / sum
+  uint64_t p_empty[kNP];            // score CTA: record r of the value CTA is free
   uint64_t v_full[kVSlots], v_empty[kVSlots], v_fixed[kVSlots];
-  uint64_t p_full[kNP];
-  uint64_t pv_prev, corr_done, o_ready, o_free;
+  uint64_t p_full[kNP];             // value CTA: record r has landed
+  uint64_t epi_req, corr_done, o_free, meta_done;
+  uint32_t req;                     // the MMA warp's request to the epilogue
   uint32_t tmem_base;
   int abort;
 };
@@ -90,26 +98,23 @@ static_assert(sizeof(Barriers) <= 1024, "barrier block too large");
 
 // shared-memory offsets from the 1024-aligned base
 constexpr uint32_t kRegion = 1024;
-__host__ __device__ constexpr uint32_t q_tile_off(int t) { return kRegion + t * kQTile; }
-__host__ __device__ constexpr uint32_t k_slot_off(int s) { return kRegion + kQSmemTiles * kQTile + s * kKSlot; }
-// score CTA staging of the P records and factors before the bulk copy
-__host__ __device__ constexpr uint32_t p_stage_off(int r) { return k_slot_off(kKSlots) + r * kPBytes; }
-__host__ __device__ constexpr uint32_t meta_stage_off(int r) {
-  return k_slot_off(kKSlots) + kNP * kPBytes + r * kMetaBytes;
-}
+// score CTA: exchange buffers, the RoPE tile of Q, the K ring
+constexpr uint32_t kXchgOff = kRegion;                       // float [2 bufs][2 halves][128]
+constexpr uint32_t kXchgBytes = 2 * 2 * 128 * 4;
+constexpr uint32_t kQRopeOff = kRegion + 3072;               // 1024-aligned
+__host__ __device__ constexpr uint32_t k_slot_off(int s) { return kQRopeOff + kQTile + s * kKSlot; }
+constexpr uint32_t kScoreSmem = k_slot_off(kKSlots);
+// value CTA: V ring, P records
 __host__ __device__ constexpr uint32_t v_slot_off(int s) { return kRegion + s * kVSlot; }
-__host__ __device__ constexpr uint32_t p_rec_off(int r) { return kRegion + kVSlots * kVSlot + r * kPBytes; }
-__host__ __device__ constexpr uint32_t meta_rec_off(int r) {
-  return kRegion + kVSlots * kVSlot + kNP * kPBytes + r * kMetaBytes;
-}
-constexpr uint32_t kScoreSmem = meta_stage_off(kNP);
-constexpr uint32_t kValueSmem = meta_rec_off(kNP);
+__host__ __device__ constexpr uint32_t rec_off(int r) { return kRegion + kVSlots * kVSlot + r * kRecBytes; }
+constexpr uint32_t kValueSmem = rec_off(kNP);
 constexpr uint32_t kSmemBytes = (kScoreSmem > kValueSmem ? kScoreSmem : kValueSmem) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(k_slot_off(0) % 1024 == 0 && p_rec_off(0) % 1024 == 0 && p_stage_off(0) % 1024 == 0,
+static_assert(kXchgBytes <= 3072 - 0, "exchange buffers");
+static_assert(kQRopeOff % 1024 == 0 && k_slot_off(0) % 1024 == 0 && rec_off(0) % 1024 == 0,
               "swizzle atoms need 1024 B");
 
-constexpr uint32_t kIdescQK = idesc_bf16(128, kPassTok, false, false);  // S[128 x 192] = Q . K^T
+__host__ __device__ constexpr uint32_t idesc_qk(int nb) { return idesc_bf16(128, 64 * nb, false, false); }
 constexpr uint32_t kIdescPV = idesc_bf16(128, 256, false, true);   // O[128x256] += P . V
 
 struct Ctx {
@@ -163,16 +168,16 @@ __device__ __forceinline__ int block_rows(const DecodeParams& p, const Segment& 
 
 // ============================================================ score CTA roles
 
-// kPassBlocks consecutive blocks of a segment form one pass (fewer at the end
-// of the segment); each pass streams its 9 column chunks through the slot
-// ring, one chunk of all the pass's blocks per slot.
+// Four consecutive blocks of a segment form one pass (fewer at the end of the
+// segment); each pass streams its 9 column chunks through the slot ring, two
+// chunks of all the pass's blocks per slot (the RoPE chunk alone).
 __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   const DecodeParams& p = *c.p;
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
   BlockCursor cur;
-  uint32_t cit = 0;
+  uint32_t fit = 0;
   bool alive = true;
   if (c.lane == 0) prefetch_tmap(tmap);
   while (alive && w.next(g)) {
@@ -189,19 +194,22 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
             atomicOr(p.err, kErrBadBlock);
         }
       }
-      for (int ch = 0; ch < 9; ++ch, ++cit) {
-        const int s = cit % kKSlots;
-        if (!warp_wait(bar_addr(c.bars->k_empty[s]), ((cit / kKSlots) & 1u) ^ 1u, c.wc)) {
+      for (int f = 0; f < kFills; ++f, ++fit) {
+        const int s = fit % kKSlots;
+        if (!warp_wait(bar_addr(c.bars->k_empty[s]), ((fit / kKSlots) & 1u) ^ 1u, c.wc)) {
           alive = false;
           break;
         }
         if (c.lane == 0) {
+          const int nch = f < 4 ? 2 : 1;
           const uint32_t full = bar_addr(c.bars->k_full[s]);
-          mbar_arrive_expect_tx(full, static_cast<uint32_t>(nb) * kChunk);
+          mbar_arrive_expect_tx(full, static_cast<uint32_t>(nb * nch) * kChunk);
           const uint32_t dst = c.base + k_slot_off(s);
+          for (int h = 0; h < nch; ++h)
 #pragma unroll
-          for (int k = 0; k < kPassBlocks; ++k)
-            if (k < nb) tma_load_2d(dst + k * kChunk, tmap, ch * 64, blk[k] * kBlock, full);
+            for (int k = 0; k < kPassBlocks; ++k)
+              if (k < nb)
+                tma_load_2d(dst + h * kPassChunk + k * kChunk, tmap, (2 * f + h) * 64, blk[k] * kBlock, full);
         }
         __syncwarp();
       }
@@ -209,7 +217,7 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   }
   // wait (bounded) for the loads this warp issued before the CTA may exit
   if (!alive) {
-    for (uint32_t k = (cit > kKSlots ? cit - kKSlots : 0); k < cit; ++k) {
+    for (uint32_t k = (fit > kKSlots ? fit - kKSlots : 0); k < fit; ++k) {
       const long long t0 = clock64();
       while (!mbar_test_wait(bar_addr(c.bars->k_full[k % kKSlots]), (k / kKSlots) & 1u) &&
              clock64() - t0 < 2000000000LL) {
@@ -218,42 +226,63 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   }
 }
 
-// The whole warp walks the segments (the walker uses warp collectives), but
-// each segment's issue loop runs in one single-thread region of lane 0:
-// issuing a slot's MMAs from a lane-0 branch that the warp enters and leaves
-// every slot measured about twice the cycles per MMA of a single-thread loop.
-__device__ bool score_mma_segment(const Ctx& c, const Segment& g, uint32_t seg, uint32_t& cit,
+// The MMAs of one slot fill: chunks 2f and 2f+1 (f < 4, A from TMEM) or the
+// RoPE chunk (f = 4, A from shared memory); four K = 16 steps per chunk.
+__device__ __forceinline__ void qk_fill(uint32_t d, uint32_t tmem, uint32_t slot, uint32_t qrope, int f,
+                                        uint32_t idesc) {
+  if (f < 4) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int ch = 2 * f + h;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts(d, tmem + kQCol + 32 * ch + 8 * kk, sw128_desc(slot + h * kPassChunk + kk * 32, 16, 1024), idesc,
+               (ch | kk) ? 1u : 0u);
+    }
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ss(d, sw128_desc(qrope + kk * 32, 16, 1024), sw128_desc(slot + kk * 32, 16, 1024), idesc, 1u);
+  }
+}
+
+// Each segment's issue loop runs in one single-thread region of lane 0.  The
+// barrier of the next slot is probed before the current slot's MMAs are
+// issued, so that the probe's latency overlaps them.
+__device__ bool score_mma_segment(const Ctx& c, const Segment& g, uint32_t seg, uint32_t& fit,
                                   uint32_t& pit) {
   const uint32_t tmem = c.tmem;
-  const uint32_t qs = c.base + q_tile_off(0);
+  const uint32_t qrope = c.base + kQRopeOff;
   const uint32_t kbase = c.base + k_slot_off(0);
   Barriers* bars = c.bars;
   if (!wait_phase(bar_addr(bars->q_ready), seg & 1u, c.wc)) return false;
   tc_fence_after();
-  for (int j = g.blk_lo; j < g.blk_hi; j += kPassBlocks, ++pit) {
-    const int sb = pit % kNS;
-    if (!wait_phase(bar_addr(bars->s_empty[sb]), ((pit / kNS) & 1u) ^ 1u, c.wc)) return false;
-    const uint32_t d = tmem + kSCol + sb * kPassTok;
-    for (int ch = 0; ch < 9; ++ch, ++cit) {
-      const int s = cit % kKSlots;
-      if (!wait_phase(bar_addr(bars->k_full[s]), (cit / kKSlots) & 1u, c.wc)) return false;
-      tc_fence_after();
-      const uint32_t tile = kbase + s * kKSlot;
-      if (ch < kQTmemChunks) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(d, tmem + kQCol + 32 * ch + 8 * kk, sw128_desc(tile + kk * 32, 16, 1024), kIdescQK,
-                 (ch | kk) ? 1u : 0u);
-      } else {
-        const uint32_t qt = qs + (ch - kQTmemChunks) * kQTile;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(d, sw128_desc(qt + kk * 32, 16, 1024), sw128_desc(tile + kk * 32, 16, 1024), kIdescQK, 1u);
-      }
+  const int npass = (g.blk_hi - g.blk_lo + kPassBlocks - 1) / kPassBlocks;
+  const int total = npass * kFills;
+  // probe of fill i of this segment
+  auto probe = [&](int i) -> bool {
+    const uint32_t k = fit + static_cast<uint32_t>(i);
+    return mbar_test_wait(bar_addr(bars->k_full[k % kKSlots]), (k / kKSlots) & 1u);
+  };
+  bool ready = probe(0);
+  for (int ps = 0; ps < npass; ++ps, ++pit) {
+    const int nb = min(kPassBlocks, g.blk_hi - g.blk_lo - ps * kPassBlocks);
+    const uint32_t idesc = idesc_qk(nb);
+    // S is single-buffered: the previous pass's softmax must have read it
+    if (!wait_phase(bar_addr(bars->s_empty), (pit & 1u) ^ 1u, c.wc)) return false;
+    tc_fence_after();
+    for (int f = 0; f < kFills; ++f) {
+      const uint32_t k = fit + static_cast<uint32_t>(ps * kFills + f);
+      const int s = k % kKSlots;
+      if (!ready && !wait_phase(bar_addr(bars->k_full[s]), (k / kKSlots) & 1u, c.wc)) return false;
+      const int nxt = ps * kFills + f + 1;
+      ready = nxt < total ? probe(nxt) : true;
+      qk_fill(tmem + kSCol, tmem, kbase + s * kKSlot, qrope, f, idesc);
       mma_commit(bar_addr(bars->k_empty[s]));
     }
-    mma_commit(bar_addr(bars->s_full[sb]));
+    mma_commit(bar_addr(bars->s_full));
   }
+  fit += static_cast<uint32_t>(total);
   mma_commit(bar_addr(bars->q_free));
   return true;
 }
@@ -263,129 +292,94 @@ __device__ void score_mma(const Ctx& c) {
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
-  uint32_t cit = 0, pit = 0, seg = 0;
+  uint32_t fit = 0, pit = 0, seg = 0;
   while (w.next(g)) {
     int ok = 1;
-    if (c.lane == 0) ok = score_mma_segment(c, g, seg, cit, pit) ? 1 : 0;
-    if (!__shfl_sync(0xffffffffu, ok, 0)) return;
+    if (c.lane == 0) ok = score_mma_segment(c, g, seg, fit, pit) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    fit = __shfl_sync(0xffffffffu, fit, 0);
+    pit = __shfl_sync(0xffffffffu, pit, 0);
+    if (!ok) return;
     ++seg;
   }
 }
 
-// Query row of sequence b for head h: columns 0..255 into TMEM lane h as 128
-// packed columns (the TS operand of the first four column chunks), columns
-// 256..575 into five swizzled [128 x 64] K-major tiles in shared memory (the
-// SS operand of the last five).
-__device__ __forceinline__ void load_q_rows(const DecodeParams& p, int b, int h, uint32_t taddr,
-                                            uint8_t* qtiles) {
+// Query row of sequence b for head h, one half per thread: half 0 writes
+// columns 0..255 into TMEM lane h (Q chunks 0-3), half 1 columns 256..511
+// (chunks 4-7) and the RoPE columns 512..575 into the swizzled shared-memory
+// tile (row h).  All global loads of a thread are issued before any store.
+__device__ __forceinline__ void load_q_half(const DecodeParams& p, int b, int h, int half, uint32_t taddr,
+                                            uint8_t* qrope) {
   const bool live = h < p.H;
   const uint4* src = reinterpret_cast<const uint4*>(p.q + (size_t(b) * p.H + (live ? h : 0)) * kRow);
   const uint4 z = make_uint4(0, 0, 0, 0);
-  const uint32_t swz = static_cast<uint32_t>(h & 7);
 #pragma unroll
-  for (int ch = 0; ch < 9; ++ch) {
-    uint4 v8[8];
+  for (int pair = 0; pair < 2; ++pair) {
+    uint4 v8[16];
 #pragma unroll
-    for (int v = 0; v < 8; ++v) v8[v] = live ? __ldg(src + ch * 8 + v) : z;
-    if (ch < kQTmemChunks) {
+    for (int v = 0; v < 16; ++v) v8[v] = live ? __ldg(src + (4 * half + 2 * pair) * 8 + v) : z;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
       uint32_t r[32];
 #pragma unroll
       for (int v = 0; v < 8; ++v) {
-        r[4 * v] = v8[v].x;
-        r[4 * v + 1] = v8[v].y;
-        r[4 * v + 2] = v8[v].z;
-        r[4 * v + 3] = v8[v].w;
+        r[4 * v] = v8[8 * hh + v].x;
+        r[4 * v + 1] = v8[8 * hh + v].y;
+        r[4 * v + 2] = v8[8 * hh + v].z;
+        r[4 * v + 3] = v8[8 * hh + v].w;
       }
-      tmem_st32(taddr + 32 * ch, r);
-    } else {
-      uint8_t* row = qtiles + (ch - kQTmemChunks) * kQTile + h * 128;
-#pragma unroll
-      for (int v = 0; v < 8; ++v)
-        *reinterpret_cast<uint4*>(row + ((static_cast<uint32_t>(v) ^ swz) << 4)) = v8[v];
+      tmem_st32(taddr + kQCol + 32 * (4 * half + 2 * pair + hh), r);
     }
   }
+  if (half == 1) {
+    const uint32_t swz = static_cast<uint32_t>(h & 7);
+    uint8_t* row = qrope + h * 128;
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      *reinterpret_cast<uint4*>(row + ((static_cast<uint32_t>(v) ^ swz) << 4)) = live ? __ldg(src + 64 + v) : z;
+  }
 }
-__device__ __forceinline__ void prefetch_q_rows_l2(const DecodeParams& p, int b, int h) {
+
+__device__ __forceinline__ void prefetch_q_row_l2(const DecodeParams& p, int b, int h) {
   if (h >= p.H) return;
   const char* src = reinterpret_cast<const char*>(p.q + (size_t(b) * p.H + h) * kRow);
 #pragma unroll
   for (int i = 0; i < 9; ++i) asm volatile("prefetch.global.L2 [%0];" ::"l"(src + 128 * i));
 }
 
-struct SoftmaxState {
-  float m_ref, l;
-};
-
-// Online softmax of one 64-token block (raw scores in sv) and its hand-off to
-// the value CTA.  Returns false if a wait gave up.
-__device__ __forceinline__ bool softmax_block(const Ctx& c, const uint32_t (&sv)[64], int nv, bool first,
-                                              float sl2, bool pos, SoftmaxState& st, uint32_t it,
-                                              int h, int q4) {
-  // block max of the scaled scores: max of s * sg with sg = sign(scale), so a
-  // negative scale needs no second code path; rows at or past nv are masked
-  const float sg = pos ? 1.f : -1.f;
-  float mr = -INFINITY;
-#pragma unroll
-  for (int t = 0; t < 64; ++t) mr = fmaxf(mr, t < nv ? __uint_as_float(sv[t]) * sg : -INFINITY);
-  const float mx = nv > 0 ? mr * sg * sl2 : -INFINITY;
-  float alpha = 1.f;
-  bool resc = false;
-  if (first) {
-    st.m_ref = mx;
-  } else if (mx > st.m_ref + kRescaleThreshold) {
-    alpha = (st.m_ref == -INFINITY) ? 0.f : ex2_approx(st.m_ref - mx);
-    st.m_ref = mx;
-    st.l *= alpha;
-    resc = true;
-  }
-  const float neg_m = st.m_ref == -INFINITY ? 0.f : -st.m_ref;
-  uint32_t pk[32];
-  float sum = 0.f;
-#pragma unroll
-  for (int t = 0; t < 32; ++t) {
-    float e0 = ex2_approx(fmaf(__uint_as_float(sv[2 * t]), sl2, neg_m));
-    float e1 = ex2_approx(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, neg_m));
-    e0 = 2 * t < nv ? e0 : 0.f;
-    e1 = 2 * t + 1 < nv ? e1 : 0.f;
-    sum += e0 + e1;
-    __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
-    pk[t] = *reinterpret_cast<uint32_t*>(&b2);
-  }
-  st.l += sum;
-
-  // P row and the per-head factors into this CTA's staging record r; the
-  // sender warps move it to the value CTA
-  const int r = it % kNP;
-  if (!warp_wait(bar_addr(c.bars->stage_empty[r]), ((it / kNP) & 1u) ^ 1u, c.wc)) return false;
-  uint8_t* prow = c.gbase + p_stage_off(r) + h * 128;
-  const uint32_t swz = static_cast<uint32_t>(h & 7);
-#pragma unroll
-  for (int ch = 0; ch < 8; ++ch)
-    *reinterpret_cast<uint4*>(prow + ((static_cast<uint32_t>(ch) ^ swz) << 4)) =
-        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-  float* meta = reinterpret_cast<float*>(c.gbase + meta_stage_off(r) + q4 * kMetaWarp);
-  meta[c.lane] = alpha;
-  meta[32 + c.lane] = st.m_ref;
-  meta[64 + c.lane] = st.l;
-  const unsigned any = __any_sync(0xffffffffu, resc);
-  if (c.lane == 0) reinterpret_cast<uint32_t*>(meta)[96] = any ? 1u : 0u;
-  mbar_arrive(bar_addr(c.bars->stage_full[r]));
+// Swap a float with the other softmax thread of the same head (same quadrant,
+// other half) through shared memory and the quadrant's exchange barrier.
+__device__ __forceinline__ bool xchg(const Ctx& c, int q4, int half, int h, uint32_t& xit, float mine,
+                                     float* other) {
+  float* buf = reinterpret_cast<float*>(c.gbase + kXchgOff) + (xit & 1u) * 256;
+  buf[half * 128 + h] = mine;
+  mbar_arrive(bar_addr(c.bars->xchg[q4]));
+  if (!warp_wait(bar_addr(c.bars->xchg[q4]), xit & 1u, c.wc)) return false;
+  *other = buf[(half ^ 1) * 128 + h];
+  ++xit;
   return true;
 }
 
 __device__ void score_softmax(const Ctx& c) {
   const DecodeParams& p = *c.p;
-  const int q4 = c.warp - 4;              // TMEM lane quadrant
+  const int q4 = c.warp & 3;              // TMEM lane quadrant (a warp reaches lanes 32*(warp%4)..)
+  const int half = (c.warp - 4) >> 2;     // blocks 2*half, 2*half+1 of each pass
   const int h = q4 * 32 + c.lane;         // head of this thread
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-  const float sl2 = p.softmax_scale * kLog2e;
+  // a zero scale (uniform attention) runs as a tiny one, so that a masked
+  // score (-inf) still gives exactly 0 (scores then differ by < 1e-27)
+  const float sl2 = p.softmax_scale != 0.f ? p.softmax_scale * kLog2e : 1e-30f;
   const bool pos = sl2 >= 0.f;
-  uint8_t* qtiles = c.gbase + q_tile_off(0);
+  const float sg = pos ? 1.f : -1.f;
+  uint8_t* qrope = c.gbase + kQRopeOff;
+  const uint32_t rec0 = map_to_rank(c.base + rec_off(0), 1);
+  const uint32_t pfull0 = map_to_rank(bar_addr(c.bars->p_full[0]), 1);
+  const uint32_t swz = static_cast<uint32_t>(h & 7);
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
   BlockCursor cur;
-  uint32_t it = 0, pit = 0, seg = 0;
+  uint32_t it = 0, pit = 0, seg = 0, xit = 0;
   bool alive = true;
   while (alive && w.next(g)) {
     cur.reset(p, g);
@@ -393,98 +387,155 @@ __device__ void score_softmax(const Ctx& c) {
       if (!warp_wait(bar_addr(c.bars->q_free), (seg - 1) & 1u, c.wc)) break;
       tc_fence_after();
     }
-    load_q_rows(p, g.b, h, c.tmem + lane_off + kQCol, qtiles);
+    load_q_half(p, g.b, h, half, c.tmem + lane_off, qrope);
     fence_proxy_async_smem();
     tmem_st_wait();
     tc_fence_before();
     mbar_arrive(bar_addr(c.bars->q_ready));
-    if (w.b < w.B && w.pre < w.e) prefetch_q_rows_l2(p, w.b, h);  // next segment's query
+    if (w.b < w.B && w.pre < w.e) prefetch_q_row_l2(p, w.b, h);  // next segment's query
 
-    SoftmaxState st{-INFINITY, 0.f};
+    float m_ref = -INFINITY, l = 0.f;
     // multi-token decode: this row's query token sees the sequence without
     // its last `short_by` tokens (0 for a plain decode)
     const int short_by = h < p.H ? p.q_len - 1 - h / p.h_per_q : 0;
     const int row_len = g.len - short_by;
-    // one block per iteration (a single inlined copy of softmax_block); the
-    // blocks of a pass share one S buffer, released after its last read
-    for (int j = g.blk_lo; j < g.blk_hi; ++j) {
-      const int k = (j - g.blk_lo) % kPassBlocks;
-      const bool last_of_pass = k == kPassBlocks - 1 || j + 1 == g.blk_hi;
-      const int sb = pit % kNS;
-      int blk;
-      const int nv = block_rows(p, g, cur, j, c.lane, &blk);
-      if (k == 0) {
-        if (!warp_wait(bar_addr(c.bars->s_full[sb]), (pit / kNS) & 1u, c.wc)) {
+    for (int j0 = g.blk_lo; j0 < g.blk_hi; j0 += kPassBlocks, ++pit) {
+      const bool first_pass = (j0 == g.blk_lo);
+      const int nb = min(kPassBlocks, g.blk_hi - j0);
+      // the two blocks of this thread in the pass (absent ones have no rows)
+      int nvr[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int kb = 2 * half + k;
+        int blk;
+        // every lane of the warp takes part in the cursor's shuffle
+        const int nv = block_rows(p, g, cur, kb < nb ? j0 + kb : j0, c.lane, &blk);
+        const int jj = j0 + kb;
+        int nr = kb < nb ? nv : 0;
+        if (p.q_len > 1) nr = max(0, min(nr, row_len - jj * kBlock));
+        nvr[k] = nr;
+      }
+      if (!warp_wait(bar_addr(c.bars->s_full), pit & 1u, c.wc)) {
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[128];
+      const uint32_t sa = c.tmem + lane_off + kSCol + 128 * half;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(sa + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * q]));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar_addr(c.bars->s_empty));
+
+      // columns at or past a block's valid count (rare: the last block of a
+      // sequence, absent blocks of a short pass) take the score -sg * inf,
+      // which no max selects; the exponentials below mask them explicitly
+      if (!__all_sync(0xffffffffu, nvr[0] == kBlock && nvr[1] == kBlock)) {
+        const uint32_t masked = __float_as_uint(-INFINITY * sg);
+#pragma unroll
+        for (int t = 0; t < 128; ++t)
+          if ((t & 63) >= nvr[t >> 6]) sv[t] = masked;
+      }
+      // pass max of the scaled scores over both threads of the head: max of
+      // s * sg with sg = sign(scale), so a negative scale needs no second
+      // code path
+      float mv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mv[u] = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < 128; ++t) mv[t & 7] = fmaxf(mv[t & 7], __uint_as_float(sv[t]) * sg);
+      const float mr = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
+                             fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+      const float mine = (nvr[0] | nvr[1]) ? mr * sg * sl2 : -INFINITY;
+      float other;
+      if (!xchg(c, q4, half, h, xit, mine, &other)) {
+        alive = false;
+        break;
+      }
+      const float mx = fmaxf(mine, other);
+      float alpha = 1.f;
+      bool resc = false;
+      if (first_pass) {
+        m_ref = mx;
+      } else if (mx > m_ref + kRescaleThreshold) {
+        alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
+        m_ref = mx;
+        l *= alpha;
+        resc = true;
+      }
+      const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
+      const unsigned any = __any_sync(0xffffffffu, resc);
+
+      // P rows of this thread's blocks straight into the value CTA's records.
+      // Columns past a block's valid count hold -sg * inf, whose exponential
+      // is exactly 0 (sl2 is never 0), so no masking is needed here.
+      const bool last_pass = j0 + kPassBlocks >= g.blk_hi;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int kb = 2 * half + k;
+        if (kb >= nb) continue;
+        const uint32_t ib = it + static_cast<uint32_t>(kb);
+        const int r = ib % kNP;
+        if (!warp_wait(bar_addr(c.bars->p_empty[r]), ((ib / kNP) & 1u) ^ 1u, c.wc)) {
           alive = false;
           break;
         }
-        tc_fence_after();
+        const uint32_t full = pfull0 + 8 * r;
+        const uint32_t rec = rec0 + r * kRecBytes;
+        // one remote arrival per warp announces the warp's bytes: each lane's
+        // P row (128) and, for a pass's first block and the segment's last,
+        // its factors (16); lane 0's rescale flag (4)
+        const bool meta = kb == 0 || (last_pass && kb == nb - 1);
+        if (c.lane == 0) mbar_arrive_expect_tx_cluster_relaxed(full, 32 * (128 + (meta ? 16 : 0)) + 4);
+        float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int t = 64 * k + 8 * ch + 2 * e;
+            const float e0 = ex2_approx(fmaf(__uint_as_float(sv[t]), sl2, neg_m));
+            const float e1 = ex2_approx(fmaf(__uint_as_float(sv[t + 1]), sl2, neg_m));
+            sum0 += e0;
+            sum1 += e1;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+            pk[e] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          st_async_v4(rec + h * 128 + ((static_cast<uint32_t>(ch) ^ swz) << 4),
+                      make_uint4(pk[0], pk[1], pk[2], pk[3]), full);
+        }
+        l += sum0 + sum1;
+        if (c.lane == 0) st_async_b32(rec + kPBytes + kMetaBytes + q4 * 4, (kb == 0 && any) ? 1u : 0u, full);
       }
-      const uint32_t sa = c.tmem + lane_off + kSCol + sb * kPassTok + 64 * k;
-      uint32_t sv[64];
-      tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_ld_wait();
-      if (last_of_pass) {
-        tc_fence_before();
-        mbar_arrive(bar_addr(c.bars->s_empty[sb]));
-        ++pit;
+      if (!alive) break;
+      // factors: the rescale factor of the pass (its first block's record)
+      // and, with the segment's last block, the running max and the sum over
+      // both threads of the head
+      float ltot = l;
+      if (last_pass) {
+        float lo;
+        if (!xchg(c, q4, half, h, xit, l, &lo)) {
+          alive = false;
+          break;
+        }
+        ltot = l + lo;
       }
-      const int nv_row = p.q_len > 1 ? max(0, min(nv, row_len - j * kBlock)) : nv;
-      if (!softmax_block(c, sv, nv_row, j == g.blk_lo, sl2, pos, st, it, h, q4)) {
-        alive = false;
-        break;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int kb = 2 * half + k;
+        if (kb >= nb || !(kb == 0 || (last_pass && kb == nb - 1))) continue;
+        const uint32_t ib = it + static_cast<uint32_t>(kb);
+        const int r = ib % kNP;
+        st_async_v4(rec0 + r * kRecBytes + kPBytes + h * 16,
+                    make_uint4(__float_as_uint(kb == 0 ? alpha : 1.f), __float_as_uint(m_ref),
+                               __float_as_uint(ltot), 0u),
+                    pfull0 + 8 * r);
       }
-      ++it;
+      if (!alive) break;
+      it += static_cast<uint32_t>(nb);
     }
     ++seg;
-  }
-  (void)alive;
-}
-
-// Sender warps (2 and 3 of the score CTA): copy each staged record into the
-// value CTA with st.async (register -> remote shared memory, bytes counted on
-// its p_full[r]) so that the slow SM-to-SM transfer overlaps the softmax of
-// the next block.
-constexpr uint32_t kRecUnits = (kPBytes + kMetaBytes) / 16;  // 16-byte units per record
-
-__device__ void score_sender(const Ctx& c) {
-  const DecodeParams& p = *c.p;
-  const int sid = (c.warp - 2) * 32 + c.lane;  // 0..63
-  const uint32_t prec0 = map_to_rank(c.base + p_rec_off(0), 1);
-  const uint32_t mrec0 = map_to_rank(c.base + meta_rec_off(0), 1);
-  const uint32_t pfull0 = map_to_rank(bar_addr(c.bars->p_full[0]), 1);
-  uint32_t my_units = 0;
-  for (uint32_t u = sid; u < kRecUnits; u += 64) ++my_units;
-  SegWalker w;
-  w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
-  Segment g;
-  uint32_t it = 0;
-  bool alive = true;
-  while (alive && w.next(g)) {
-    for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
-      const int r = it % kNP;
-      if (!warp_wait(bar_addr(c.bars->stage_full[r]), (it / kNP) & 1u, c.wc) ||
-          !warp_wait(bar_addr(c.bars->p_empty[r]), ((it / kNP) & 1u) ^ 1u, c.wc)) {
-        alive = false;
-        break;
-      }
-      const uint32_t fullr = pfull0 + 8 * r;
-      mbar_arrive_expect_tx_cluster_relaxed(fullr, my_units * 16);
-      const uint8_t* pst = c.gbase + p_stage_off(r);
-      const uint8_t* mst = c.gbase + meta_stage_off(r);
-      for (uint32_t u = sid; u < kRecUnits; u += 64) {
-        if (u < kPBytes / 16) {
-          const uint4 v = *reinterpret_cast<const uint4*>(pst + u * 16);
-          st_async_v4(prec0 + r * kPBytes + u * 16, v, fullr);
-        } else {
-          const uint32_t m = u - kPBytes / 16;
-          const uint4 v = *reinterpret_cast<const uint4*>(mst + m * 16);
-          st_async_v4(mrec0 + r * kMetaBytes + m * 16, v, fullr);
-        }
-      }
-      mbar_arrive(bar_addr(c.bars->stage_empty[r]));
-    }
   }
   // drain: every record handed to the value CTA has been released, so no
   // remote arrival on this CTA is still pending when it exits
@@ -575,36 +626,50 @@ __device__ void value_fixup(const Ctx& c) {
   }
 }
 
-// As for the score MMA warp: each segment's issue loop is one single-thread
-// region of lane 0.
+// As for the score MMA warp: each segment's issue loop runs in one
+// single-thread region of lane 0, and the next slot's barrier is probed
+// before the current slot's MMAs are issued.  The epilogue warps act only on
+// requests: a rescale of O before a record's PV, and the final output after
+// the segment's last PV (kReqFinal | record), each posted in `req` with a
+// plain arrival on epi_req plus a commit (the MMAs issued so far are done).
+constexpr uint32_t kReqFinal = 0x80000000u;
+
+__device__ __forceinline__ void post_request(const Ctx& c, uint32_t req) {
+  *reinterpret_cast<volatile uint32_t*>(&c.bars->req) = req;
+  mbar_arrive(bar_addr(c.bars->epi_req));
+  mma_commit(bar_addr(c.bars->epi_req));
+}
+
 __device__ bool value_mma_segment(const Ctx& c, const Segment& g, uint32_t seg, uint32_t& it,
                                   uint32_t& vit, uint32_t& ncorr) {
   if (seg > 0) {
     if (!wait_phase(bar_addr(c.bars->o_free), (seg - 1) & 1u, c.wc)) return false;
     tc_fence_after();
   }
+  bool ready = mbar_test_wait(bar_addr(c.bars->v_fixed[vit % kVSlots]), (vit / kVSlots) & 1u);
   for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
     const int r = it % kNP;
     if (!wait_phase(bar_addr(c.bars->p_full[r]), (it / kNP) & 1u, c.wc)) return false;
     const bool first = (j == g.blk_lo);
-    const uint8_t* meta = c.gbase + meta_rec_off(r);
-    uint32_t any = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) any |= reinterpret_cast<const uint32_t*>(meta + q * kMetaWarp)[96];
+    const bool last = (j == g.blk_hi - 1);
+    const uint32_t* flags = reinterpret_cast<const uint32_t*>(c.gbase + rec_off(r) + kPBytes + kMetaBytes);
+    const uint32_t any = flags[0] | flags[1] | flags[2] | flags[3];
     if (any && !first) {
       // hand O over for rescaling once every MMA issued so far (the previous
-      // block's PV) has completed, and take it back when rescaled
-      mma_commit(bar_addr(c.bars->pv_prev));
+      // blocks' PV) has completed, and take it back when rescaled
+      post_request(c, static_cast<uint32_t>(r));
       if (!wait_phase(bar_addr(c.bars->corr_done), ncorr & 1u, c.wc)) return false;
       ++ncorr;
+      tc_fence_after();
     }
     fence_proxy_async_smem();
-    const uint32_t pa = c.base + p_rec_off(r);
+    const uint32_t pa = c.base + rec_off(r);
     for (int n = 0; n < 2; ++n, ++vit) {
       const int s = vit % kVSlots;
-      if (!wait_phase(bar_addr(c.bars->v_full[s]), (vit / kVSlots) & 1u, c.wc)) return false;
-      if (!wait_phase(bar_addr(c.bars->v_fixed[s]), (vit / kVSlots) & 1u, c.wc)) return false;
-      tc_fence_after();
+      // v_fixed completes after v_full (the fixup warp waits v_full first)
+      if (!ready && !wait_phase(bar_addr(c.bars->v_fixed[s]), (vit / kVSlots) & 1u, c.wc)) return false;
+      const uint32_t nx = vit + 1;
+      ready = mbar_test_wait(bar_addr(c.bars->v_fixed[nx % kVSlots]), (nx / kVSlots) & 1u);
       const uint32_t va = c.base + v_slot_off(s);
 #pragma unroll
       for (int k = 0; k < kBlock / 16; ++k)
@@ -612,8 +677,10 @@ __device__ bool value_mma_segment(const Ctx& c, const Segment& g, uint32_t seg, 
                sw128_desc(va + k * 2048, kChunk, 1024), kIdescPV, (k > 0 || !first) ? 1u : 0u);
       mma_commit(bar_addr(c.bars->v_empty[s]));
     }
-    mma_commit_mc(bar_addr(c.bars->p_empty[r]), 0x1);
-    if (j == g.blk_hi - 1) mma_commit(bar_addr(c.bars->o_ready));  // O final for this segment
+    if (last)
+      post_request(c, kReqFinal | static_cast<uint32_t>(r));  // the epilogue releases the record
+    else
+      mma_commit_mc(bar_addr(c.bars->p_empty[r]), 0x1);
   }
   return true;
 }
@@ -632,96 +699,96 @@ __device__ void value_mma(const Ctx& c) {
   }
 }
 
+// Thread = (head h, latent half): the rescales and the final normalisation
+// of O's 256 columns [256 * half, 256 * half + 256) of TMEM lane h, on the
+// MMA warp's requests.
 __device__ void value_epilogue(const Ctx& c) {
   const DecodeParams& p = *c.p;
-  const int q4 = c.warp - 4;
+  const int q4 = c.warp & 3;
+  const int half = (c.warp - 4) >> 2;
   const int h = q4 * 32 + c.lane;
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+  const uint32_t ocol = 256 * half;
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
-  uint32_t it = 0, seg = 0, ncorr = 0;
+  uint32_t nreq = 0, nfinal = 0;
   while (w.next(g)) {
-    float m_fin = -INFINITY, l_fin = 0.f;
-    for (int j = g.blk_lo; j < g.blk_hi; ++j, ++it) {
-      const int r = it % kNP;
-      if (!warp_wait(bar_addr(c.bars->p_full[r]), (it / kNP) & 1u, c.wc)) return;
-      const uint8_t* meta = c.gbase + meta_rec_off(r);
-      const float alpha = reinterpret_cast<const float*>(meta + q4 * kMetaWarp)[c.lane];
-      uint32_t any = 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) any |= reinterpret_cast<const uint32_t*>(meta + q * kMetaWarp)[96];
-      const bool first = (j == g.blk_lo);
-      const bool last = (j == g.blk_hi - 1);
-      if (last) {
-        m_fin = reinterpret_cast<const float*>(meta + q4 * kMetaWarp)[32 + c.lane];
-        l_fin = reinterpret_cast<const float*>(meta + q4 * kMetaWarp)[64 + c.lane];
-      }
-      __syncwarp();
-      if (c.lane == 0) mbar_arrive_remote(bar_addr(c.bars->p_empty[r]), 0);
-      if (any && !first) {
-        // the MMA warp hands O over (pv_prev) once the previous block's PV is done
-        if (!warp_wait(bar_addr(c.bars->pv_prev), ncorr & 1u, c.wc)) return;
-        ++ncorr;
-        tc_fence_after();
+    for (;;) {
+      if (!warp_wait(bar_addr(c.bars->epi_req), nreq & 1u, c.wc)) return;
+      ++nreq;
+      tc_fence_after();
+      const uint32_t req = *reinterpret_cast<volatile uint32_t*>(&c.bars->req);
+      const uint8_t* rec = c.gbase + rec_off(static_cast<int>(req & 0xffu));
+      const float4 meta = *reinterpret_cast<const float4*>(rec + kPBytes + h * 16);
+      if (!(req & kReqFinal)) {
+        const float alpha = meta.x;
 #pragma unroll 1
-        for (int ch = 0; ch < 16; ++ch) {
+        for (int ch = 0; ch < 8; ++ch) {
           uint32_t v[32];
-          tmem_ld32(c.tmem + lane_off + 32 * ch, v);
+          tmem_ld32(c.tmem + lane_off + ocol + 32 * ch, v);
           tmem_ld_wait();
 #pragma unroll
           for (int t = 0; t < 32; ++t) v[t] = __float_as_uint(__uint_as_float(v[t]) * alpha);
-          tmem_st32(c.tmem + lane_off + 32 * ch, v);
+          tmem_st32(c.tmem + lane_off + ocol + 32 * ch, v);
         }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar_addr(c.bars->corr_done));
+        continue;
       }
-      if (last) {
-        if (!warp_wait(bar_addr(c.bars->o_ready), seg & 1u, c.wc)) return;
-        tc_fence_after();
-        const bool live = h < p.H;
-        const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
-        const float lse = l_fin > 0.f ? (m_fin + log2f(l_fin)) * 0.6931471805599453f : -INFINITY;
+      // final: O / l and lse (or the fp32 piece of a cut sequence).  The
+      // record goes back to the score CTA once all eight warps have read it.
+      const float m_fin = meta.y, l_fin = meta.z;
+      __syncwarp();
+      if (c.lane == 0) mbar_arrive(bar_addr(c.bars->meta_done));
+      if (c.warp == 4) {
+        if (!warp_wait(bar_addr(c.bars->meta_done), nfinal & 1u, c.wc)) return;
+        if (c.lane == 0) mbar_arrive_remote(bar_addr(c.bars->p_empty[req & 0xffu]), 0);
+      }
+      ++nfinal;
+      const bool live = h < p.H;
+      const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
+      const float lse = l_fin > 0.f ? (m_fin + log2f(l_fin)) * 0.6931471805599453f : -INFINITY;
 #pragma unroll 1
-        for (int ch = 0; ch < 16; ++ch) {
-          uint32_t v[32];
-          tmem_ld32(c.tmem + lane_off + 32 * ch, v);
-          tmem_ld_wait();
-          if (!live) continue;
-          if (g.slot < 0) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t(g.b) * p.H + h) * kDc + 32 * ch);
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(c.tmem + lane_off + ocol + 32 * ch, v);
+        tmem_ld_wait();
+        if (!live) continue;
+        const int col = ocol + 32 * ch;
+        if (g.slot < 0) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t(g.b) * p.H + h) * kDc + col);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t w4[4];
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w4[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]) * inv,
-                                                          __uint_as_float(v[8 * q + 2 * e + 1]) * inv);
-                w4[e] = *reinterpret_cast<uint32_t*>(&b2);
-              }
-              dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]) * inv,
+                                                        __uint_as_float(v[8 * q + 2 * e + 1]) * inv);
+              w4[e] = *reinterpret_cast<uint32_t*>(&b2);
             }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(p.o_part + (size_t(g.slot) * p.H + h) * kDc + 32 * ch);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(__uint_as_float(v[4 * q]) * inv, __uint_as_float(v[4 * q + 1]) * inv,
-                                   __uint_as_float(v[4 * q + 2]) * inv, __uint_as_float(v[4 * q + 3]) * inv);
+            dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.o_part + (size_t(g.slot) * p.H + h) * kDc + col);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(v[4 * q]) * inv, __uint_as_float(v[4 * q + 1]) * inv,
+                                 __uint_as_float(v[4 * q + 2]) * inv, __uint_as_float(v[4 * q + 3]) * inv);
         }
-        tc_fence_before();
-        mbar_arrive(bar_addr(c.bars->o_free));
-        if (live) {
-          if (g.slot < 0)
-            p.lse[size_t(g.b) * p.H + h] = lse;
-          else
-            p.lse_part[size_t(g.slot) * p.H + h] = lse;
-        }
-        if (h == 0 && g.first_of_seq) p.seq_info[g.b] = seq_info_for(g, w);
       }
+      tc_fence_before();
+      mbar_arrive(bar_addr(c.bars->o_free));
+      if (live && half == 0) {
+        if (g.slot < 0)
+          p.lse[size_t(g.b) * p.H + h] = lse;
+        else
+          p.lse_part[size_t(g.slot) * p.H + h] = lse;
+      }
+      if (h == 0 && half == 0 && g.first_of_seq) p.seq_info[g.b] = seq_info_for(g, w);
+      break;
     }
-    ++seg;
   }
 }
 
@@ -743,27 +810,24 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
       mbar_init(smem_u32(&bars->k_full[s]), 1);
       mbar_init(smem_u32(&bars->k_empty[s]), 1);
     }
-    for (int s = 0; s < kNS; ++s) {
-      mbar_init(smem_u32(&bars->s_full[s]), 1);
-      mbar_init(smem_u32(&bars->s_empty[s]), 128);
-    }
-    mbar_init(smem_u32(&bars->q_ready), 128);
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->s_empty), 256);       // every softmax thread
+    mbar_init(smem_u32(&bars->q_ready), 256);
     mbar_init(smem_u32(&bars->q_free), 1);
+    for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&bars->xchg[q]), 64);  // two warps
     for (int r = 0; r < kNP; ++r) {
-      mbar_init(smem_u32(&bars->p_empty[r]), 1 + 4);  // PV commit + 4 epilogue warps
-      mbar_init(smem_u32(&bars->p_full[r]), 64);      // every sender thread (+ st.async bytes)
-      mbar_init(smem_u32(&bars->stage_full[r]), 128); // every softmax thread
-      mbar_init(smem_u32(&bars->stage_empty[r]), 64); // every sender thread
+      mbar_init(smem_u32(&bars->p_empty[r]), 1);      // PV commit, or the epilogue (segment end)
+      mbar_init(smem_u32(&bars->p_full[r]), 4);       // the four softmax warps of one half
     }
     for (int s = 0; s < kVSlots; ++s) {
       mbar_init(smem_u32(&bars->v_full[s]), 1);
       mbar_init(smem_u32(&bars->v_empty[s]), 1);
       mbar_init(smem_u32(&bars->v_fixed[s]), 1);
     }
-    mbar_init(smem_u32(&bars->pv_prev), 1);
-    mbar_init(smem_u32(&bars->corr_done), 128);
-    mbar_init(smem_u32(&bars->o_ready), 1);
-    mbar_init(smem_u32(&bars->o_free), 128);
+    mbar_init(smem_u32(&bars->epi_req), 2);         // request word posted + commit
+    mbar_init(smem_u32(&bars->corr_done), 256);
+    mbar_init(smem_u32(&bars->o_free), 256);
+    mbar_init(smem_u32(&bars->meta_done), 8);        // every epilogue warp read the final record
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -781,21 +845,23 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
   c.gbase = gbase;
   c.bars = bars;
   c.tmem = bars->tmem_base;
-  c.wc = WaitCtx{p.spin_limit, p.err, &bars->abort};
+  c.wc = WaitCtx{p.spin_limit, p.err, &bars->abort, p.err + 1};
   c.engine = blockIdx.x >> 1;
   c.warp = warp;
   c.lane = lane;
 
-  if (rank == 0) {
-    if (warp == 0) score_tma(c, &tmap);
-    else if (warp == 1) score_mma(c);
-    else if (warp <= 3) score_sender(c);
-    else score_softmax(c);
+  if (warp < 4) {
+    if (rank == 0) {
+      if (warp == 0) score_tma(c, &tmap);
+      else if (warp == 1) score_mma(c);
+    } else {
+      if (warp == 0) value_tma(c, &tmap);
+      else if (warp == 1) value_mma(c);
+      else if (warp == 2) value_fixup(c);
+    }
   } else {
-    if (warp == 0) value_tma(c, &tmap);
-    else if (warp == 1) value_mma(c);
-    else if (warp == 2) value_fixup(c);
-    else if (warp >= 4) value_epilogue(c);
+    if (rank == 0) score_softmax(c);
+    else value_epilogue(c);
   }
 
   __syncthreads();

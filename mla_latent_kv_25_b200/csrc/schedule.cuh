@@ -51,7 +51,7 @@ struct SegWalker {
   int len;
   int count;        // segments returned so far
 
-  __device__ void init(const int32_t* sl, int B_, int maxb, int P_, int p_) {
+  __device__ __noinline__ void init(const int32_t* sl, int B_, int maxb, int P_, int p_) {
     seq_lens = sl;
     B = B_;
     max_blocks = maxb;
@@ -99,7 +99,7 @@ struct SegWalker {
   }
 
   // Next segment; false when the engine's range is exhausted.
-  __device__ bool next(Segment& g) {
+  __device__ __noinline__ bool next(Segment& g) {
     if (b >= B || pre >= e) return false;
     long long lo = s > pre ? s : pre;
     long long hi = e < pre + nb ? e : pre + nb;

@@ -86,6 +86,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded-wait context: every wait gives up after `limit` SM clock cycles,
 // records kErrTimeout in the workspace error word and raises the CTA's abort
 // flag, which makes every other waiter of the CTA give up too.
+// Polling of a wait: kSpinPolls back-to-back probes, then one probe per
+// kPollSleepNs nanoseconds of sleep.
+constexpr uint32_t kSpinPolls = 16;
+constexpr uint32_t kPollSleepNs = 32;
+
 struct WaitCtx {
   long long limit;
   uint32_t* err;
@@ -127,13 +132,15 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // decode pipeline's hand-offs costs more than the issue slots polling takes.
 // Arguments by value: a reference would force the caller's context into
 // local memory, and every asm statement with a "memory" clobber (all the
-// barrier, TMA and MMA wrappers here) would then reload it.  Inlined: a call
-// out of a region that runs under setmaxnreg cannot be register-allocated.
-static __device__ __forceinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, long long limit,
+// barrier, TMA and MMA wrappers here) would then reload it.
+static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, long long limit,
                                                     uint32_t* err, volatile int* abort, uint32_t* where) {
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_test_wait(bar, parity)) return true;
+    // after a short spin, poll every few tens of nanoseconds: a spinning
+    // thread takes issue slots from the warps that share its scheduler
+    if (i > kSpinPolls) __nanosleep(kPollSleepNs);
     if ((i & 63u) == 0) {
       if (*abort) return false;
       if (clock64() - t0 > limit) {
@@ -153,11 +160,38 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const 
   return wait_phase_slow(bar, parity, w.limit, w.err, w.abort, w.where);
 }
 
-// Whole-warp wait: every lane waits (each takes its own acquire); the warp
-// proceeds only if every lane saw the phase complete.
+// Whole-warp wait: lane 0 polls (one poller per warp keeps the barrier unit
+// free for the threads that issue TMA and MMA work), then every lane takes
+// its own acquire with one probe of the completed phase.
+// Inlined: the softmax waits with a head's scores live in registers, which a
+// call would have to save and restore.
+__device__ __forceinline__ bool warp_wait_slow(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  const bool lead = (threadIdx.x & 31) == 0;
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    bool done = false;
+    if (lead) done = mbar_test_wait(bar, parity);
+    if (__shfl_sync(0xffffffffu, done ? 1 : 0, 0)) break;
+    if (i > kSpinPolls) __nanosleep(kPollSleepNs);
+    if ((i & 63u) == 0) {
+      if (*w.abort) return false;
+      if (clock64() - t0 > w.limit) {
+        if (lead) {
+          atomicOr(w.err, kErrTimeout);
+          if (w.where != nullptr && atomicCAS(w.where, 0u, bar | 0x80000000u) == 0u)
+            w.where[1] = (blockIdx.x << 8) | (threadIdx.x >> 5);
+          *w.abort = 1;
+        }
+        return false;
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
+}
+
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
-  const bool ok = wait_phase(bar, parity, w);
-  return __all_sync(0xffffffffu, ok);
+  if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+  return warp_wait_slow(bar, parity, w);
 }
 
 // ------------------------------------------------------------------ TMA / bulk copies
@@ -241,18 +275,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_cluster_relaxed(uint32_t b
                    bar_cluster),
                "r"(bytes)
                : "memory");
-}
-
-// Register reallocation between warpgroups (all four warps of a warpgroup
-// execute it).  The sum over warpgroups must stay within the registers the
-// block was launched with (threads x registers per thread at launch).
-template <uint32_t N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // 2^x on the special-function unit (flush-to-zero for tiny results).

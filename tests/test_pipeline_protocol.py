@@ -12,13 +12,15 @@ model; completing later cannot create a cycle that the model misses, since
 no role waits on anything but barrier phases.
 
 The model is a transcription: a change to the kernel's waits, arrivals,
-ring sizes or barrier counts must be made here too.
+ring sizes or barrier counts must be made here too.  Rescale flags are drawn
+per block (the kernel raises them only on a pass's first block; the protocol
+is the same).
 """
 import random
 
 import pytest
 
-K_SLOTS, N_S, N_REC, V_SLOTS, PASS = 3, 2, 3, 5, 3
+K_SLOTS, FILLS, N_REC, V_SLOTS, PASS = 3, 5, 4, 4, 4
 
 
 class Bar:
@@ -39,7 +41,18 @@ class Bar:
         return ok
 
 
+def _passes(lo, hi):
+    j = lo
+    while j < hi:
+        nb = min(PASS, hi - j)
+        yield j, nb
+        j += nb
+
+
 def roles(segs, rescale, k_slots, n_rec):
+    """The kernel's roles as generators: score CTA (TMA, QK MMA, the two
+    softmax halves of 128 threads), value CTA (TMA, fixup warp, PV MMA, the
+    eight epilogue warps)."""
     B = {}
 
     def bar(name, count):
@@ -47,75 +60,74 @@ def roles(segs, rescale, k_slots, n_rec):
 
     for i in range(k_slots):
         bar(f"k_full{i}", 1); bar(f"k_empty{i}", 1)
-    for i in range(N_S):
-        bar(f"s_full{i}", 1); bar(f"s_empty{i}", 128)
-    bar("q_ready", 128); bar("q_free", 1)
+    bar("s_full", 1); bar("s_empty", 256)
+    bar("q_ready", 256); bar("q_free", 1)
+    bar("xchg", 2)                                   # one quadrant's two warps, one per half
     for i in range(n_rec):
-        bar(f"stage_full{i}", 128); bar(f"stage_empty{i}", 64)   # score CTA staging
-        bar(f"p_full{i}", 64); bar(f"p_empty{i}", 5)             # value CTA record / its release
+        bar(f"p_full{i}", 4)                         # the four warps of the writing half
+        bar(f"p_empty{i}", 1)                        # PV commit, or the epilogue at a segment end
     for i in range(V_SLOTS):
         bar(f"v_full{i}", 1); bar(f"v_empty{i}", 1); bar(f"v_fixed{i}", 1)
-    bar("pv_prev", 1); bar("corr_done", 128); bar("o_ready", 1); bar("o_free", 128)
+    bar("epi_req", 2); bar("corr_done", 256); bar("o_free", 256); bar("meta_done", 8)
 
     def wait(name, parity, phase=None):
         return ("wait", name, parity, phase)
 
     def score_tma():
-        cit = 0
+        fit = 0
         for lo, hi in segs:
-            for _ in range(lo, hi, PASS):
-                for _ch in range(9):
-                    s = cit % k_slots
-                    yield wait(f"k_empty{s}", ((cit // k_slots) & 1) ^ 1, cit // k_slots - 1)
+            for _j, _nb in _passes(lo, hi):
+                for _f in range(FILLS):
+                    s = fit % k_slots
+                    yield wait(f"k_empty{s}", ((fit // k_slots) & 1) ^ 1, fit // k_slots - 1)
                     B[f"k_full{s}"].arrive()
-                    cit += 1
+                    fit += 1
 
     def score_mma():
-        cit = pit = 0
+        fit = pit = 0
         for seg, (lo, hi) in enumerate(segs):
             yield wait("q_ready", seg & 1, seg)
-            for _ in range(lo, hi, PASS):
-                sb = pit % N_S
-                yield wait(f"s_empty{sb}", ((pit // N_S) & 1) ^ 1, pit // N_S - 1)
-                for _ch in range(9):
-                    s = cit % k_slots
-                    yield wait(f"k_full{s}", (cit // k_slots) & 1, cit // k_slots)
+            for _j, _nb in _passes(lo, hi):
+                yield wait("s_empty", (pit & 1) ^ 1, pit - 1)
+                for _f in range(FILLS):
+                    s = fit % k_slots
+                    yield wait(f"k_full{s}", (fit // k_slots) & 1, fit // k_slots)
                     B[f"k_empty{s}"].arrive()
-                    cit += 1
-                B[f"s_full{sb}"].arrive()
+                    fit += 1
+                B["s_full"].arrive()
                 pit += 1
             B["q_free"].arrive()
 
-    def softmax():
-        it = pit = 0
+    def softmax(half):
+        it = pit = xit = 0
         for seg, (lo, hi) in enumerate(segs):
             if seg > 0:
                 yield wait("q_free", (seg - 1) & 1, seg - 1)
             B["q_ready"].arrive(128)
-            for j in range(lo, hi):
-                k = (j - lo) % PASS
-                sb = pit % N_S
-                if k == 0:
-                    yield wait(f"s_full{sb}", (pit // N_S) & 1, pit // N_S)
-                if k == PASS - 1 or j + 1 == hi:
-                    B[f"s_empty{sb}"].arrive(128)
-                    pit += 1
-                r = it % n_rec
-                yield wait(f"stage_empty{r}", ((it // n_rec) & 1) ^ 1, it // n_rec - 1)
-                B[f"stage_full{r}"].arrive(128)
-                it += 1
-
-    def sender():
-        it = 0
-        for lo, hi in segs:
-            for _ in range(lo, hi):
-                r = it % n_rec
-                yield wait(f"stage_full{r}", (it // n_rec) & 1, it // n_rec)
-                yield wait(f"p_empty{r}", ((it // n_rec) & 1) ^ 1, it // n_rec - 1)
-                B[f"p_full{r}"].arrive(64)        # st.async bytes land with the arrivals
-                B[f"stage_empty{r}"].arrive(64)
-                it += 1
-        for k in range(max(0, it - n_rec), it):  # drain: every record released
+            for j0, nb in _passes(lo, hi):
+                yield wait("s_full", pit & 1, pit)
+                B["s_empty"].arrive(128)
+                pit += 1
+                B["xchg"].arrive()
+                yield wait("xchg", xit & 1, xit)
+                xit += 1
+                mine = []
+                for k in range(2):
+                    kb = 2 * half + k
+                    if kb >= nb:
+                        continue
+                    ib = it + kb
+                    r = ib % n_rec
+                    yield wait(f"p_empty{r}", ((ib // n_rec) & 1) ^ 1, ib // n_rec - 1)
+                    mine.append(r)
+                if j0 + PASS >= hi:                  # last pass: the sums are exchanged
+                    B["xchg"].arrive()
+                    yield wait("xchg", xit & 1, xit)
+                    xit += 1
+                for r in mine:                       # a record is full once its bytes landed
+                    B[f"p_full{r}"].arrive(4)
+                it += nb
+        for k in range(max(0, it - n_rec), it):      # drain: every record released
             yield wait(f"p_empty{k % n_rec}", (k // n_rec) & 1, k // n_rec)
 
     def value_tma():
@@ -147,38 +159,41 @@ def roles(segs, rescale, k_slots, n_rec):
                 r = it % n_rec
                 yield wait(f"p_full{r}", (it // n_rec) & 1, it // n_rec)
                 if rescale[it] and j != lo:
-                    B["pv_prev"].arrive()
+                    B["epi_req"].arrive(2)           # request posted + commit
                     yield wait("corr_done", ncorr & 1, ncorr)
                     ncorr += 1
                 for _n in range(2):
                     s = vit % V_SLOTS
-                    yield wait(f"v_full{s}", (vit // V_SLOTS) & 1, vit // V_SLOTS)
                     yield wait(f"v_fixed{s}", (vit // V_SLOTS) & 1, vit // V_SLOTS)
                     B[f"v_empty{s}"].arrive()
                     vit += 1
-                B[f"p_empty{r}"].arrive()          # commit multicast to the score CTA
                 if j == hi - 1:
-                    B["o_ready"].arrive()
+                    B["epi_req"].arrive(2)           # final request; the epilogue releases r
+                else:
+                    B[f"p_empty{r}"].arrive()        # commit multicast to the score CTA
                 it += 1
 
     def epilogue():
-        it = ncorr = 0
+        it = nreq = nfinal = 0
         for seg, (lo, hi) in enumerate(segs):
             for j in range(lo, hi):
                 r = it % n_rec
-                yield wait(f"p_full{r}", (it // n_rec) & 1, it // n_rec)
-                B[f"p_empty{r}"].arrive(4)              # remote, one per warp
                 if rescale[it] and j != lo:
-                    yield wait("pv_prev", ncorr & 1, ncorr)
-                    ncorr += 1
-                    B["corr_done"].arrive(128)
+                    yield wait("epi_req", nreq & 1, nreq)
+                    nreq += 1
+                    B["corr_done"].arrive(256)
                 if j == hi - 1:
-                    yield wait("o_ready", seg & 1, seg)
-                    B["o_free"].arrive(128)
+                    yield wait("epi_req", nreq & 1, nreq)
+                    nreq += 1
+                    B["meta_done"].arrive(8)
+                    yield wait("meta_done", nfinal & 1, nfinal)
+                    nfinal += 1
+                    B[f"p_empty{r}"].arrive()        # remote, by one warp
+                    B["o_free"].arrive(256)
                 it += 1
 
-    procs = dict(score_tma=score_tma(), score_mma=score_mma(), softmax=softmax(),
-                 sender=sender(), value_tma=value_tma(), fixup=fixup(),
+    procs = dict(score_tma=score_tma(), score_mma=score_mma(), softmax0=softmax(0),
+                 softmax1=softmax(1), value_tma=value_tma(), fixup=fixup(),
                  value_mma=value_mma(), epilogue=epilogue())
     return B, procs
 
@@ -238,13 +253,12 @@ def test_protocol_finishes_in_every_interleaving(k_slots):
 
 
 def test_model_finds_a_planted_deadlock():
-    """Planted fault: the value CTA's MMA releases records only after the
-    epilogue's arrivals would need a fifth arrival that never comes (a
-    record count of 6 instead of 5): the sender then waits for good."""
+    """Planted fault: the record-release barrier expects two arrivals where
+    the value CTA gives one: the softmax then waits for good."""
     orig = Bar.__init__
 
     def planted(self, name, count):
-        orig(self, name, 6 if name.startswith("p_empty") else count)
+        orig(self, name, 2 if name.startswith("p_empty") else count)
 
     Bar.__init__ = planted
     try:
