@@ -12,12 +12,16 @@
 //   w1    MMA: S = Q K^T for 256 tokens at once          MN-major), N = 256 per instruction
 //         (N = 256); Q columns 0..511 in TMEM      w2    zero V rows past seq_len
 //         (TS), the RoPE columns in shared memory  w4-11 thread = (head, latent half): O
-//   w4-11 softmax, thread = (head, half pass):            rescale when a max moved; final
-//         reads its 128 S columns at once (so the        O / l and lse, or an fp32 piece
-//         next pass's QK can start), online              of a cut sequence
-//         softmax in fp32, and sends P (bf16) and
-//         the per-head factors straight into the
-//         value CTA's shared memory (st.async)
+//   w4-11 softmax, thread = (head, 2 of the            rescale when a max moved; final
+//         pass's 4 blocks: warps 4-7 take blocks         O / l and lse, or an fp32 piece
+//         0 and 2, warps 8-11 blocks 1 and 3, so         of a cut sequence
+//         that records reach the value CTA in
+//         the order it consumes them): reads its
+//         128 S columns at once (so the next
+//         pass's QK can start), online softmax in
+//         fp32, and sends P (bf16) and the
+//         per-head factors straight into the value
+//         CTA's shared memory (st.async)
 //
 // Why this shape (measured on B200): a single-CTA tcgen05.mma costs about
 // 120-135 cycles to issue whatever its N up to 192, so only N = 256 runs the
@@ -25,8 +29,9 @@
 // with A in TMEM, the PV at ~129); an mbarrier probe between MMAs stalls the
 // issue stream unless it is issued ahead of the MMAs it guards, so every MMA
 // loop polls the next stage's barrier before issuing the current stage; the
-// SM-to-SM hand-off peaks at ~21 bytes per clock, enough for one 16 KB P tile
-// per block when 256 threads issue the stores.
+// SM-to-SM hand-off peaks at ~21 bytes per clock, and only for whole 32-byte
+// sectors: a lane's 16-byte store alone moves half as much, so lanes pair up
+// to write both halves of a sector.
 //
 // Heads are the M = 128 dimension of both contractions (padded with zero query
 // rows for H < 128).  The running max of a head moves only when a pass's max
@@ -58,7 +63,7 @@ constexpr int kPassTok = kPassBlocks * kBlock;
 constexpr int kKSlots = 3;                      // score CTA: ring of two-chunk slots
 constexpr int kFills = 5;                       // slot fills per pass: chunks {0,1} {2,3} {4,5} {6,7} {8}
 constexpr int kVSlots = 4;                      // value CTA: ring of [64 x 256] half-block slots
-constexpr int kNP = 4;                          // P records in flight (value CTA)
+constexpr int kNP = 5;                          // P records in flight (value CTA)
 
 constexpr uint32_t kChunk = 64 * 128;           // [64 rows x 64 bf16] swizzled (one block, one chunk)
 constexpr uint32_t kPassChunk = kPassBlocks * kChunk;  // one column chunk of a pass [256 x 64]
@@ -363,7 +368,7 @@ __device__ __forceinline__ bool xchg(const Ctx& c, int q4, int half, int h, uint
 __device__ void score_softmax(const Ctx& c) {
   const DecodeParams& p = *c.p;
   const int q4 = c.warp & 3;              // TMEM lane quadrant (a warp reaches lanes 32*(warp%4)..)
-  const int half = (c.warp - 4) >> 2;     // blocks 2*half, 2*half+1 of each pass
+  const int half = (c.warp - 4) >> 2;     // blocks half, half + 2 of each pass
   const int h = q4 * 32 + c.lane;         // head of this thread
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
   // a zero scale (uniform attention) runs as a tiny one, so that a masked
@@ -406,7 +411,7 @@ __device__ void score_softmax(const Ctx& c) {
       int nvr[2];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        const int kb = 2 * half + k;
+        const int kb = half + 2 * k;
         int blk;
         // every lane of the warp takes part in the cursor's shuffle
         const int nv = block_rows(p, g, cur, kb < nb ? j0 + kb : j0, c.lane, &blk);
@@ -421,9 +426,10 @@ __device__ void score_softmax(const Ctx& c) {
       }
       tc_fence_after();
       uint32_t sv[128];
-      const uint32_t sa = c.tmem + lane_off + kSCol + 128 * half;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(sa + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * q]));
+      for (int q = 0; q < 4; ++q)
+        tmem_ld32(c.tmem + lane_off + kSCol + 64 * half + 128 * (q >> 1) + 32 * (q & 1),
+                  *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * q]));
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(bar_addr(c.bars->s_empty));
@@ -440,13 +446,24 @@ __device__ void score_softmax(const Ctx& c) {
       // pass max of the scaled scores over both threads of the head: max of
       // s * sg with sg = sign(scale), so a negative scale needs no second
       // code path
-      float mv[8];
+      float mr;
+      if (pos) {
+        float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mv[u] = -INFINITY;
+        for (int t = 0; t < 128; t += 8)
 #pragma unroll
-      for (int t = 0; t < 128; ++t) mv[t & 7] = fmaxf(mv[t & 7], __uint_as_float(sv[t]) * sg);
-      const float mr = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
-                             fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+          for (int u = 0; u < 4; ++u)
+            mv[u] = fmax3(mv[u], __uint_as_float(sv[t + 2 * u]), __uint_as_float(sv[t + 2 * u + 1]));
+        mr = fmax3(fmaxf(mv[0], mv[1]), mv[2], mv[3]);
+      } else {
+        float mv[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+#pragma unroll
+        for (int t = 0; t < 128; t += 8)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            mv[u] = fmin3(mv[u], __uint_as_float(sv[t + 2 * u]), __uint_as_float(sv[t + 2 * u + 1]));
+        mr = -fmin3(fminf(mv[0], mv[1]), mv[2], mv[3]);
+      }
       const float mine = (nvr[0] | nvr[1]) ? mr * sg * sl2 : -INFINITY;
       float other;
       if (!xchg(c, q4, half, h, xit, mine, &other)) {
@@ -473,7 +490,7 @@ __device__ void score_softmax(const Ctx& c) {
       const bool last_pass = j0 + kPassBlocks >= g.blk_hi;
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        const int kb = 2 * half + k;
+        const int kb = half + 2 * k;
         if (kb >= nb) continue;
         const uint32_t ib = it + static_cast<uint32_t>(kb);
         const int r = ib % kNP;
@@ -489,24 +506,44 @@ __device__ void score_softmax(const Ctx& c) {
         const bool meta = kb == 0 || (last_pass && kb == nb - 1);
         if (c.lane == 0) mbar_arrive_expect_tx_cluster_relaxed(full, 32 * (128 + (meta ? 16 : 0)) + 4);
         float sum0 = 0.f, sum1 = 0.f;
+        // chunks 2t and 2t+1 of a row share a 32-byte sector of the record;
+        // lanes 2i and 2i+1 trade one chunk each so that every store writes
+        // a whole sector (row 2i, then row 2i+1)
+        const bool odd = c.lane & 1;
+        const uint32_t row_a = static_cast<uint32_t>(h & ~1), row_b = row_a + 1;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t pk[4];
+        for (int tp = 0; tp < 4; ++tp) {
+          uint32_t pk[2][4];
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int t = 64 * k + 16 * tp + 8 * u + 2 * e;
+              const float e0 = ex2_approx(fmaf(__uint_as_float(sv[t]), sl2, neg_m));
+              const float e1 = ex2_approx(fmaf(__uint_as_float(sv[t + 1]), sl2, neg_m));
+              sum0 += e0;
+              sum1 += e1;
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+              pk[u][e] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+          uint32_t d1[4], d2[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int t = 64 * k + 8 * ch + 2 * e;
-            const float e0 = ex2_approx(fmaf(__uint_as_float(sv[t]), sl2, neg_m));
-            const float e1 = ex2_approx(fmaf(__uint_as_float(sv[t + 1]), sl2, neg_m));
-            sum0 += e0;
-            sum1 += e1;
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
-            pk[e] = *reinterpret_cast<uint32_t*>(&b2);
+            const uint32_t got = __shfl_xor_sync(0xffffffffu, odd ? pk[0][e] : pk[1][e], 1);
+            d1[e] = odd ? got : pk[0][e];   // row 2i: chunk 2t (even lane), 2t+1 (odd lane)
+            d2[e] = odd ? pk[1][e] : got;   // row 2i+1: chunk 2t (even lane), 2t+1 (odd lane)
           }
-          st_async_v4(rec + h * 128 + ((static_cast<uint32_t>(ch) ^ swz) << 4),
-                      make_uint4(pk[0], pk[1], pk[2], pk[3]), full);
+          const uint32_t chl = static_cast<uint32_t>(2 * tp) | (odd ? 1u : 0u);
+          st_async_v4(rec + row_a * 128 + ((chl ^ (row_a & 7)) << 4), make_uint4(d1[0], d1[1], d1[2], d1[3]), full);
+          st_async_v4(rec + row_b * 128 + ((chl ^ (row_b & 7)) << 4), make_uint4(d2[0], d2[1], d2[2], d2[3]), full);
         }
         l += sum0 + sum1;
         if (c.lane == 0) st_async_b32(rec + kPBytes + kMetaBytes + q4 * 4, (kb == 0 && any) ? 1u : 0u, full);
+        // a pass's first block carries the pass's rescale factor; unless it
+        // is also the segment's last block, its factors are final now
+        if (kb == 0 && !(last_pass && nb == 1))
+          st_async_v4(rec + kPBytes + h * 16,
+                      make_uint4(__float_as_uint(alpha), __float_as_uint(m_ref), __float_as_uint(l), 0u), full);
       }
       if (!alive) break;
       // factors: the rescale factor of the pass (its first block's record)
@@ -523,8 +560,8 @@ __device__ void score_softmax(const Ctx& c) {
       }
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        const int kb = 2 * half + k;
-        if (kb >= nb || !(kb == 0 || (last_pass && kb == nb - 1))) continue;
+        const int kb = half + 2 * k;
+        if (!(last_pass && kb == nb - 1)) continue;
         const uint32_t ib = it + static_cast<uint32_t>(kb);
         const int r = ib % kNP;
         st_async_v4(rec0 + r * kRecBytes + kPBytes + h * 16,

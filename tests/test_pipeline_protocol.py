@@ -20,7 +20,7 @@ import random
 
 import pytest
 
-K_SLOTS, FILLS, N_REC, V_SLOTS, PASS = 3, 5, 4, 4, 4
+K_SLOTS, FILLS, N_REC, V_SLOTS, PASS = 3, 5, 5, 4, 4
 
 
 class Bar:
@@ -111,21 +111,25 @@ def roles(segs, rescale, k_slots, n_rec):
                 B["xchg"].arrive()
                 yield wait("xchg", xit & 1, xit)
                 xit += 1
-                mine = []
+                last_pass = j0 + PASS >= hi
+                final = None
                 for k in range(2):
-                    kb = 2 * half + k
+                    kb = half + 2 * k                # blocks half and half + 2
                     if kb >= nb:
                         continue
                     ib = it + kb
                     r = ib % n_rec
                     yield wait(f"p_empty{r}", ((ib // n_rec) & 1) ^ 1, ib // n_rec - 1)
-                    mine.append(r)
-                if j0 + PASS >= hi:                  # last pass: the sums are exchanged
+                    if last_pass and kb == nb - 1:
+                        final = r                    # its factors wait for the sums
+                    else:
+                        B[f"p_full{r}"].arrive(4)    # a record is full once its bytes landed
+                if last_pass:                        # last pass: the sums are exchanged
                     B["xchg"].arrive()
                     yield wait("xchg", xit & 1, xit)
                     xit += 1
-                for r in mine:                       # a record is full once its bytes landed
-                    B[f"p_full{r}"].arrive(4)
+                if final is not None:
+                    B[f"p_full{final}"].arrive(4)
                 it += nb
         for k in range(max(0, it - n_rec), it):      # drain: every record released
             yield wait(f"p_empty{k % n_rec}", (k // n_rec) & 1, k // n_rec)
