@@ -61,6 +61,8 @@ typedef enum {
 #define MLA_DEVERR_BAD_BLOCK   0x1u  /* a block_table entry needed by seq_lens is < 0 or >= num_blocks */
 #define MLA_DEVERR_SEQ_TOO_LONG 0x2u /* seq_lens[b] > 64 * max_blocks_per_seq or < 0 */
 #define MLA_DEVERR_TIMEOUT     0x4u  /* a bounded wait inside a kernel gave up; the kernel exited */
+#define MLA_DEVERR_BAD_PIECES  0x8u  /* decode: split-KV bookkeeping out of range (internal error);
+                                        the affected rows read out = 0, lse = NaN */
 
 /*
  * mla_absorb_q - fold the key up-projection into the query ("Empirical Gains":
@@ -106,8 +108,8 @@ mla_status_t mla_absorb_get_error(void *stream, uint32_t *err_bits);
 size_t mla_decode_workspace_bytes(int B, int H, int num_splits);
 
 /*
- * mla_decode_fp8_workspace_bytes - workspace bytes that let mla_decode run an
- * fp8 cache on the tensor cores: mla_decode_workspace_bytes(B, H, num_splits)
+ * mla_decode_fp8_workspace_bytes - workspace bytes that let mla_decode widen
+ * the whole batch of an fp8 cache at once: mla_decode_workspace_bytes(B, H, num_splits)
  * rounded up to 256, plus a scratch block table (4 * B * max_blocks_per_seq
  * bytes, rounded up to 256) and a widened bf16 copy of the blocks the batch
  * reads (73,728 bytes per table entry: B * max_blocks_per_seq blocks of
@@ -127,15 +129,17 @@ size_t mla_decode_fp8_workspace_bytes(int B, int H, int max_blocks_per_seq, int 
  * k_rope:      fp8 cache only: bf16 [num_blocks,64,64]; must be NULL for bf16.
  * block_scale: fp8 cache only: f32 [num_blocks], c_kv = e4m3(code) * scale;
  *              must be NULL for bf16.
- *              The fp8 cache is decoded one of two ways, chosen by
- *              workspace_bytes.  With at least
+ *              The fp8 cache runs in two kernels: the first writes the rows
+ *              a group of sequences reads as bf16
+ *              [bf16(e4m3(code) * scale) | k_rope] into the workspace (round
+ *              to nearest even: relative error <= 2^-9 per element), the
+ *              tensor-core decode then reads them as a bf16 cache.  With
  *              mla_decode_fp8_workspace_bytes(B, H, max_blocks_per_seq,
- *              num_splits) bytes, a first kernel writes the rows the batch
- *              reads as bf16 [bf16(e4m3(code) * scale) | k_rope] into the
- *              workspace (round to nearest even: relative error <= 2^-9 per
- *              element), and the tensor-core decode reads them.  With less
- *              (but at least mla_decode_workspace_bytes), a CUDA-core decode
- *              reads the codes directly, in fp32, about 20x slower.
+ *              num_splits) bytes the group is the whole batch; with less,
+ *              the call runs the largest groups of consecutive sequences (and
+ *              if need be fewer split-KV engines) that fit, one after the
+ *              other on `stream`; MLA_ERR_WORKSPACE_TOO_SMALL when not even
+ *              one sequence on one engine fits.
  * block_table: int32 [B, max_blocks_per_seq]; logical block j of sequence b is
  *              physical block block_table[b*max_blocks_per_seq + j].  Entries
  *              at j >= ceil(seq_lens[b]/64) are never read (pad with -1).
@@ -162,6 +166,9 @@ size_t mla_decode_fp8_workspace_bytes(int B, int H, int max_blocks_per_seq, int 
  * Checked on the device (recorded as error bits, the offending rows are
  * skipped): block ids in range, seq_lens in range.  Every internal wait is
  * bounded; on expiry the kernel records MLA_DEVERR_TIMEOUT and exits cleanly.
+ * While MLA_DEVERR_TIMEOUT is set in the workspace's error word (it stays set
+ * until mla_get_device_error reads it), every row a call writes reads out = 0,
+ * lse = NaN, so that no result of an incomplete decode is ever returned.
  */
 mla_status_t mla_decode(const void *q, mla_cache_dtype_t cache_dtype, const void *cache,
                         const void *k_rope, const float *block_scale,
@@ -230,16 +237,28 @@ mla_status_t mla_get_device_error(void *workspace, void *stream, uint32_t *err_b
  * up the array's address on that device; make it before any stream capture.
  * All calls on a device share the array and it keeps the last call's
  * contents: calls that overlap on the GPU race, so serialise them.  Nothing
- * in it needs clearing between calls.  Device-side error bits are recorded
- * in the array but not reported.  An fp8 cache takes the tensor-core route
- * when mla_decode_fp8_workspace_bytes(...) fits in the 40 MiB, else the
- * CUDA-core decode (see mla_decode).  Allocates and frees no device memory.
+ * in it needs clearing between calls.  Device-side error bits accumulate in
+ * the array's error word; read and clear them with
+ * mla_decode_noalloc_get_error (while MLA_DEVERR_TIMEOUT is set there, calls
+ * write out = 0, lse = NaN, as mla_decode does).  An fp8 cache is widened in
+ * the array: the whole batch when mla_decode_fp8_workspace_bytes(...) fits in
+ * the 40 MiB, else in groups of sequences (see mla_decode).  Allocates and
+ * frees no device memory.
  */
 mla_status_t mla_decode_noalloc(const void *q, mla_cache_dtype_t cache_dtype, const void *cache,
                                 const void *k_rope, const float *block_scale,
                                 const int32_t *block_table, const int32_t *seq_lens, int B, int H,
                                 int num_blocks, int max_blocks_per_seq, float softmax_scale,
                                 void *out, float *lse, int num_splits, void *stream);
+
+/*
+ * mla_decode_noalloc_get_error - mla_get_device_error for the built-in
+ * scratch of mla_decode_noalloc on the current device: waits for `stream`,
+ * stores the accumulated MLA_DEVERR_* bits in *err_bits and clears them.
+ * MLA_ERR_INVALID_ARG if err_bits is NULL, MLA_ERR_CUDA if the scratch
+ * cannot be located or the copy fails.
+ */
+mla_status_t mla_decode_noalloc_get_error(void *stream, uint32_t *err_bits);
 
 /*
  * mla_cache_append - write the rows of T new tokens into the paged bf16 cache

@@ -26,13 +26,14 @@ MLA_CACHE_FP8_E4M3 = 1
 DEVERR_BAD_BLOCK = 0x1
 DEVERR_SEQ_TOO_LONG = 0x2
 DEVERR_TIMEOUT = 0x4
+DEVERR_BAD_PIECES = 0x8
 
 # every symbol include/mla.h declares
 EXPORTS = ("mla_absorb_q", "mla_absorb_o", "mla_absorb_get_error", "mla_cache_append",
            "mla_cache_quantize_fp8", "mla_cache_get_error", "mla_set_wait_limit", "mla_decode_multi",
            "mla_decode_workspace_bytes", "mla_decode_fp8_workspace_bytes", "mla_decode",
            "mla_combine", "mla_get_device_error", "mla_status_string", "mla_num_sms",
-           "mla_decode_noalloc", "mla_last_error_string")
+           "mla_decode_noalloc", "mla_decode_noalloc_get_error", "mla_last_error_string")
 
 
 class MLAError(RuntimeError):
@@ -94,6 +95,8 @@ def load():
         L.mla_decode_noalloc.restype = i32
         L.mla_decode_noalloc.argtypes = [vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                          ctypes.c_float, vp, vp, i32, vp]
+        L.mla_decode_noalloc_get_error.restype = i32
+        L.mla_decode_noalloc_get_error.argtypes = [vp, vp]
         _lib = L
         return L
 
@@ -323,6 +326,15 @@ def mla_combine(o_part, lse_part, out, lse, stream=None):
     _check("mla_combine", load().mla_combine(_ptr(o_part), _ptr(lse_part), B, H, S, _ptr(out),
                                              _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def mla_decode_noalloc_get_error(stream=None) -> int:
+    """Synchronise the stream, return and clear the error bits of the
+    built-in scratch of mla_decode_noalloc (current device)."""
+    v = ctypes.c_uint32(0)
+    _check("mla_decode_noalloc_get_error",
+           load().mla_decode_noalloc_get_error(_stream(stream), ctypes.byref(v)))
+    return int(v.value)
 
 
 def mla_get_device_error(workspace, stream=None) -> int:

@@ -295,6 +295,26 @@ mla_status_t mla_absorb_get_error(void* stream, uint32_t* err_bits) {
 
 namespace {
 
+// One decode launch and its merge over a bf16 cache: p's split-KV scratch
+// (error word, per-sequence records, partial results) is laid out at the
+// start of `workspace` for p.B sequences and p.P engines.
+mla_status_t decode_group(DecodeParams p, void* workspace, cudaStream_t st) {
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  const WsLayout ws = ws_layout(p.B, p.H, p.P);
+  p.err = reinterpret_cast<uint32_t*>(wsb);
+  p.seq_info = reinterpret_cast<int4*>(wsb + ws.seq_info);
+  p.lse_part = reinterpret_cast<float*>(wsb + ws.lse_part);
+  p.o_part = reinterpret_cast<float*>(wsb + ws.o_part);
+  CUtensorMap tmap;
+  if (!encode_bf16_map(&tmap, p.cache, uint64_t(p.num_blocks) * kBlock, kRow, kRow * 2))
+    return fail_with("tensor map encoding failed");
+  cudaError_t e = launch_decode_sm100(p, tmap, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_merge_pieces(p.seq_lens, p.B, p.max_blocks, p.H, p.P, p.seq_info, p.lse_part, p.o_part,
+                          p.out, p.lse, p.err, st);
+  return status_of(e);
+}
+
 // Shared by mla_decode (q_len = 1) and mla_decode_multi: the q_len query
 // tokens of a sequence are q_len * H rows of one engine's contraction.
 mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype, const void* cache,
@@ -324,15 +344,12 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
     return MLA_ERR_INVALID_ARG;
   const int P = resolve_engines(num_splits, B);
   if (P < 1) return fail_with("no streaming multiprocessor count for the current device");
-  const WsLayout ws = ws_layout(B, rows, P);
-  if (workspace_bytes < ws.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < ws_layout(B, rows, P).total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  uint8_t* wsb = static_cast<uint8_t*>(workspace);
   DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.cache = cache;
-  p.k_rope = static_cast<const __nv_bfloat16*>(k_rope);
-  p.block_scale = block_scale;
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.B = B;
@@ -344,45 +361,55 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
   p.softmax_scale = softmax_scale;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  p.err = reinterpret_cast<uint32_t*>(wsb);
-  p.seq_info = reinterpret_cast<int4*>(wsb + ws.seq_info);
-  p.lse_part = reinterpret_cast<float*>(wsb + ws.lse_part);
-  p.o_part = reinterpret_cast<float*>(wsb + ws.o_part);
   p.P = P;
   p.spin_limit = g_decode_wait_limit.load();
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!fp8) return decode_group(p, workspace, st);
 
-  cudaError_t e;
-  // The fp8 cache takes the tensor-core decode through its widened bf16 copy
-  // when the workspace has room for it, else the CUDA-core decode.
-  const long long wide_blocks = static_cast<long long>(B) * max_blocks_per_seq;
-  const WideLayout wide = wide_layout(ws.total, B, max_blocks_per_seq);
-  const bool widen = fp8 && wide_blocks <= kMaxWideBlocks && workspace_bytes >= wide.total;
-  if (widen) {
+  // The fp8 cache: each group of sequences is widened to bf16 rows in the
+  // workspace, then decoded like a bf16 cache.  One group when the workspace
+  // holds the whole batch's widened copy (mla_decode_fp8_workspace_bytes);
+  // else the largest groups (and, if need be, fewer split-KV engines) that fit.
+  int Bg = B, Pg = P;
+  for (;;) {
+    const long long wide_blocks = static_cast<long long>(Bg) * max_blocks_per_seq;
+    if (wide_blocks <= kMaxWideBlocks &&
+        wide_layout(ws_layout(Bg, rows, Pg).total, Bg, max_blocks_per_seq).total <= workspace_bytes)
+      break;
+    if (Pg > 1) {
+      Pg = (Pg + 1) / 2;
+    } else if (Bg > 1) {
+      Bg = (Bg + 1) / 2;
+      Pg = resolve_engines(num_splits, Bg);
+    } else {
+      return MLA_ERR_WORKSPACE_TOO_SMALL;
+    }
+  }
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  for (int b0 = 0; b0 < B; b0 += Bg) {
+    const int nb = min(Bg, B - b0);
+    const int pg = min(Pg, resolve_engines(num_splits, nb));
+    const WideLayout wide = wide_layout(ws_layout(nb, rows, pg).total, nb, max_blocks_per_seq);
     int32_t* wide_table = reinterpret_cast<int32_t*>(wsb + wide.table);
     __nv_bfloat16* wide_cache = reinterpret_cast<__nv_bfloat16*>(wsb + wide.cache);
-    e = launch_fp8_widen(static_cast<const uint8_t*>(cache), p.k_rope, block_scale, block_table,
-                         seq_lens, B, max_blocks_per_seq, num_blocks, wide_table, wide_cache, p.err,
-                         device_sms(), st);
+    const int32_t* table_g = block_table + static_cast<size_t>(b0) * max_blocks_per_seq;
+    cudaError_t e = launch_fp8_widen(static_cast<const uint8_t*>(cache),
+                                     static_cast<const __nv_bfloat16*>(k_rope), block_scale, table_g,
+                                     seq_lens + b0, nb, max_blocks_per_seq, num_blocks, wide_table,
+                                     wide_cache, reinterpret_cast<uint32_t*>(wsb), device_sms(), st);
     if (e != cudaSuccess) return cuda_fail(e);
-    p.cache = wide_cache;
-    p.k_rope = nullptr;
-    p.block_scale = nullptr;
-    p.block_table = wide_table;
-    p.num_blocks = static_cast<int>(wide_blocks);
+    DecodeParams g = p;
+    g.q = p.q + static_cast<size_t>(b0) * rows * kRow;
+    g.out = p.out + static_cast<size_t>(b0) * rows * kDc;
+    g.lse = p.lse + static_cast<size_t>(b0) * rows;
+    g.seq_lens = seq_lens + b0;
+    g.B = nb;
+    g.P = pg;
+    g.cache = wide_cache;
+    g.block_table = wide_table;
+    g.num_blocks = static_cast<int>(static_cast<long long>(nb) * max_blocks_per_seq);
+    if (mla_status_t s = decode_group(g, workspace, st); s != MLA_OK) return s;
   }
-  if (!fp8 || widen) {
-    CUtensorMap tmap;
-    if (!encode_bf16_map(&tmap, p.cache, uint64_t(p.num_blocks) * kBlock, kRow, kRow * 2))
-      return fail_with("tensor map encoding failed");
-    e = launch_decode_sm100(p, tmap, st);
-  } else {
-    e = launch_decode_simt(p, fp8, st);
-  }
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = launch_merge_pieces(seq_lens, B, max_blocks_per_seq, rows, p.seq_info, p.lse_part, p.o_part,
-                          p.out, p.lse, p.err, st);
-  return status_of(e);
+  return MLA_OK;
 }
 
 }  // namespace

@@ -68,13 +68,16 @@ __device__ __forceinline__ void merge_row(int n, LseAt lse_at, OAt o_at, __nv_bf
 
 // grid (B, ceil(H / kRowsPerCta)); warp w merges head blockIdx.y * kRowsPerCta + w.
 __global__ void __launch_bounds__(kMergeThreads)
-merge_pieces_kernel(const int32_t* __restrict__ seq_lens, int max_blocks, int H,
+merge_pieces_kernel(const int32_t* __restrict__ seq_lens, int max_blocks, int H, int P,
                     const int4* __restrict__ seq_info, const float* __restrict__ lse_part,
                     const float* __restrict__ o_part, __nv_bfloat16* __restrict__ out,
                     float* __restrict__ lse, uint32_t* __restrict__ err) {
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31;
   const int h = blockIdx.y * kRowsPerCta + (threadIdx.x >> 5);
+  // a decode that gave up (timeout) left seq_info and the pieces incomplete:
+  // every row then reads out = 0, lse = NaN instead of stale workspace data
+  const bool aborted = (*reinterpret_cast<volatile uint32_t*>(err) & kErrTimeout) != 0;
   int L = seq_lens[b];
   if (L < 0 || L > max_blocks * kBlock) {
     if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(err, kErrSeqTooLong);
@@ -82,16 +85,30 @@ merge_pieces_kernel(const int32_t* __restrict__ seq_lens, int max_blocks, int H,
   }
   if (h >= H) return;
   __nv_bfloat16* row = out + (size_t(b) * H + h) * kDc;
-  if (L == 0) {
+  auto fill = [&](float lse_value) {
     uint4* dst = reinterpret_cast<uint4*>(row + lane * 16);
     dst[0] = make_uint4(0u, 0u, 0u, 0u);
     dst[1] = make_uint4(0u, 0u, 0u, 0u);
-    if (lane == 0) lse[size_t(b) * H + h] = -INFINITY;
+    if (lane == 0) lse[size_t(b) * H + h] = lse_value;
+  };
+  if (aborted) {
+    fill(NAN);
+    return;
+  }
+  if (L == 0) {
+    fill(-INFINITY);
     return;
   }
   const int4 info = seq_info[b];
-  if (info.w != kSeqCut) return;  // written directly by its engine
+  if (info.w == kSeqWhole) return;  // written directly by its engine
   const int p0 = info.x, p1 = info.y, slot0 = info.z;
+  // the pieces of a cut sequence are engines p0..p1 (slot0 for p0's piece,
+  // 2p for the others); anything else is inconsistent bookkeeping
+  if (info.w != kSeqCut || p0 < 0 || p1 >= P || p0 > p1 || slot0 < 0 || slot0 >= 2 * P) {
+    if (lane == 0) atomicOr(err, kErrBadPieces);
+    fill(NAN);
+    return;
+  }
   const int n = p1 - p0 + 1;
   auto slot_of = [&](int i) { return i == 0 ? slot0 : 2 * (p0 + i); };
   auto lse_at = [&](int i) { return lse_part[size_t(slot_of(i)) * H + h]; };
@@ -112,12 +129,12 @@ combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_p
 
 }  // namespace
 
-cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H,
+cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H, int P,
                                 const int4* seq_info, const float* lse_part, const float* o_part,
                                 __nv_bfloat16* out, float* lse, uint32_t* err,
                                 cudaStream_t stream) {
   dim3 grid(B, (H + kRowsPerCta - 1) / kRowsPerCta);
-  merge_pieces_kernel<<<grid, kMergeThreads, 0, stream>>>(seq_lens, max_blocks, H, seq_info,
+  merge_pieces_kernel<<<grid, kMergeThreads, 0, stream>>>(seq_lens, max_blocks, H, P, seq_info,
                                                           lse_part, o_part, out, lse, err);
   return cudaGetLastError();
 }

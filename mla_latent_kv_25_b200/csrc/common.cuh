@@ -18,6 +18,7 @@ constexpr int kMaxHeads = 128;
 constexpr uint32_t kErrBadBlock = 0x1u;
 constexpr uint32_t kErrSeqTooLong = 0x2u;
 constexpr uint32_t kErrTimeout = 0x4u;
+constexpr uint32_t kErrBadPieces = 0x8u;
 
 // ---------------------------------------------------------------------------
 // Workspace layout (all offsets 256-byte aligned):

@@ -379,7 +379,6 @@ __device__ void score_softmax(const Ctx& c) {
   uint8_t* qrope = c.gbase + kQRopeOff;
   const uint32_t rec0 = map_to_rank(c.base + rec_off(0), 1);
   const uint32_t pfull0 = map_to_rank(bar_addr(c.bars->p_full[0]), 1);
-  const uint32_t swz = static_cast<uint32_t>(h & 7);
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;

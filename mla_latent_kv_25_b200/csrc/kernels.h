@@ -10,9 +10,7 @@ namespace mla {
 
 struct DecodeParams {
   const __nv_bfloat16* q;          // [B,H,576] (H = rows per sequence)
-  const void* cache;               // bf16 [NB,64,576] | u8 [NB,64,512]
-  const __nv_bfloat16* k_rope;     // fp8 cache: [NB,64,64]
-  const float* block_scale;        // fp8 cache: [NB]
+  const void* cache;               // bf16 [NB,64,576]
   const int32_t* block_table;      // [B,max_blocks]
   const int32_t* seq_lens;         // [B]
   int B, H, num_blocks, max_blocks;
@@ -31,10 +29,6 @@ struct DecodeParams {
   int q_len, h_per_q;
 };
 
-// CUDA-core decode (any H multiple of 16); fp8: cache is E4M3.  Used for the
-// fp8 cache when the workspace has no room for the widened bf16 copy.
-cudaError_t launch_decode_simt(const DecodeParams& p, bool fp8, cudaStream_t stream);
-
 // Tensor-core decode (bf16 cache): clusters of two CTAs, one engine each.
 // `tmap` is a 2-D tiled map over the cache viewed as [num_blocks*64, 576]
 // bf16 with a 64 x 64 box and 128-byte swizzle.
@@ -42,7 +36,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, 
 size_t decode_sm100_smem_bytes();
 int decode_sm100_max_clusters();
 
-cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H,
+cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H, int P,
                                 const int4* seq_info, const float* lse_part, const float* o_part,
                                 __nv_bfloat16* out, float* lse, uint32_t* err,
                                 cudaStream_t stream);

@@ -15,23 +15,22 @@
 //     (mla_decode_workspace_bytes(B, H, num_splits)) exceeds it is rejected
 //     with MLA_ERR_WORKSPACE_TOO_SMALL and nothing is launched.  At H = 128
 //     and the automatic split count of a B200 the need is about 39 MB.
-//   - The first call on a device looks up the array's device address on that
-//     device (cudaGetSymbolAddress with the device current); make that first
-//     call before any stream capture.
+//   - Every call looks up the array's device address on the current device
+//     (cudaGetSymbolAddress), so the address stays right after a device reset;
+//     make the first call on a device (which loads the module) before any
+//     stream capture.
 //   - Every call on a device shares the array, which keeps the last call's
 //     contents.  Calls whose executions overlap on the GPU (different streams,
 //     or host threads racing) race on it; serialise them.
 //   - Nothing in the array needs clearing between calls: every value a call
 //     reads (per-sequence records, partial results) is written earlier in the
 //     same call.  The array starts zeroed when the library is loaded; its
-//     error word accumulates device-side error bits of all calls and is not
-//     reported by this entry point (invalid block ids are still skipped).
-//   - An fp8 cache runs on the tensor cores (through its widened bf16 copy)
-//     when mla_decode_fp8_workspace_bytes fits in the array, else on the
-//     CUDA-core decode.
+//     error word accumulates device-side error bits of all calls until
+//     mla_decode_noalloc_get_error reads and clears it.
+//   - An fp8 cache is widened to bf16 rows in the array: the whole batch at
+//     once when mla_decode_fp8_workspace_bytes fits in it, else in groups of
+//     sequences (as mla_decode does with a smaller workspace).
 //   - No device memory is allocated or freed by this entry point.
-#include <mutex>
-
 #include "../../include/mla.h"
 #include "common.cuh"
 
@@ -41,23 +40,12 @@ constexpr size_t kNoAllocScratchBytes = size_t(40) << 20;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
-
-// Device address of the scratch array on the current device (looked up once
-// per device).  Returns nullptr on failure.
+// Device address of the scratch array on the current device.  Returns
+// nullptr on failure.
 void* scratch_for_current_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> g(g_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
-      return nullptr;
-    g_scratch_ptr[dev] = ptr;
-  }
-  return g_scratch_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  return ptr;
 }
 
 }  // namespace
@@ -76,4 +64,11 @@ extern "C" mla_status_t mla_decode_noalloc(const void* q, mla_cache_dtype_t cach
   return mla_decode(q, cache_dtype, cache, k_rope, block_scale, block_table, seq_lens, B, H,
                     num_blocks, max_blocks_per_seq, softmax_scale, out, lse, ws,
                     kNoAllocScratchBytes, num_splits, stream);
+}
+
+extern "C" mla_status_t mla_decode_noalloc_get_error(void* stream, uint32_t* err_bits) {
+  if (err_bits == nullptr) return MLA_ERR_INVALID_ARG;
+  void* ws = scratch_for_current_device();
+  if (ws == nullptr) return MLA_ERR_CUDA;
+  return mla_get_device_error(ws, stream, err_bits);
 }

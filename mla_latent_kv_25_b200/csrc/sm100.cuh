@@ -141,7 +141,7 @@ static __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parit
     // after a short spin, poll every few tens of nanoseconds: a spinning
     // thread takes issue slots from the warps that share its scheduler
     if (i > kSpinPolls) __nanosleep(kPollSleepNs);
-    if ((i & 63u) == 0) {
+    if ((i & 7u) == 0) {
       if (*abort) return false;
       if (clock64() - t0 > limit) {
         atomicOr(err, kErrTimeout);
@@ -173,7 +173,7 @@ __device__ __forceinline__ bool warp_wait_slow(uint32_t bar, uint32_t parity, co
     if (lead) done = mbar_test_wait(bar, parity);
     if (__shfl_sync(0xffffffffu, done ? 1 : 0, 0)) break;
     if (i > kSpinPolls) __nanosleep(kPollSleepNs);
-    if ((i & 63u) == 0) {
+    if ((i & 7u) == 0) {
       if (*w.abort) return false;
       if (clock64() - t0 > w.limit) {
         if (lead) {

@@ -44,11 +44,12 @@ def test_error_codes_agree_across_header_kernels_and_binding():
     bits = {n: int(v, 16) for n, v in re.findall(r"#define (MLA_DEVERR_[A-Z_]+)\s+0x([0-9a-fA-F]+)u", hdr)}
     assert bits == {"MLA_DEVERR_BAD_BLOCK": binding.DEVERR_BAD_BLOCK,
                     "MLA_DEVERR_SEQ_TOO_LONG": binding.DEVERR_SEQ_TOO_LONG,
-                    "MLA_DEVERR_TIMEOUT": binding.DEVERR_TIMEOUT}
+                    "MLA_DEVERR_TIMEOUT": binding.DEVERR_TIMEOUT,
+                    "MLA_DEVERR_BAD_PIECES": binding.DEVERR_BAD_PIECES}
     common = open(os.path.join(ROOT, "mla_latent_kv_25_b200", "csrc", "common.cuh")).read()
     kern = {n: int(v, 16) for n, v in re.findall(r"constexpr uint32_t (kErr[A-Za-z]+) = 0x([0-9a-fA-F]+)u;", common)}
     assert kern == {"kErrBadBlock": bits["MLA_DEVERR_BAD_BLOCK"], "kErrSeqTooLong": bits["MLA_DEVERR_SEQ_TOO_LONG"],
-                    "kErrTimeout": bits["MLA_DEVERR_TIMEOUT"]}
+                    "kErrTimeout": bits["MLA_DEVERR_TIMEOUT"], "kErrBadPieces": bits["MLA_DEVERR_BAD_PIECES"]}
 
 
 def test_status_strings():

@@ -55,14 +55,14 @@ def test_sharp_softmax():
     check_full(w, 5, what="sharp")
 
 
-@pytest.mark.parametrize("route", ["tensor", "cuda-core"])
+@pytest.mark.parametrize("route", ["whole", "groups"])
 def test_fp8_cache_small(route):
-    """The fp8 cache through the widened bf16 copy (workspace sized by
-    mla_decode_fp8_workspace_bytes) and through the CUDA-core decode (a
-    workspace of mla_decode_workspace_bytes, no room for the copy)."""
+    """The fp8 cache widened for the whole batch at once (workspace sized by
+    mla_decode_fp8_workspace_bytes) and one sequence at a time (a workspace
+    with room for one sequence's widened copy only)."""
     w = inputs.make("fp8", B=3, H=32, L=[200, 64, 1], seed=24, q_std=2.0, extra_blocks=2)
     d = binding.to_device(w)
-    ws = None if route == "tensor" else binding.alloc_workspace(w.B, w.H, 3)
+    ws = None if route == "whole" else binding.alloc_workspace(1, w.H, 3, fp8_max_blocks=w.max_blocks)
     out, lse, ws = binding.decode_device(d, w.softmax_scale, num_splits=3, workspace=ws)
     assert binding.mla_get_device_error(ws) == 0
     ro, rl = oracle.decode_workload(w)
@@ -70,15 +70,23 @@ def test_fp8_cache_small(route):
     assert_close(to_np(lse).reshape(-1), rl, f"fp8 {route} lse")
 
 
-def test_fp8_routes_agree_on_a_ragged_batch():
+def test_fp8_groups_agree_on_a_ragged_batch():
+    """Whole-batch widening and groups of two sequences (3 groups, the last
+    one short) give the oracle's result; a workspace without room for one
+    sequence's widened copy is rejected before any launch."""
     w = inputs.make("fp8", B=5, H=64, L=[1, 700, 65, 64, 2000], seed=33, q_std=3.0, extra_blocks=3)
     d = binding.to_device(w)
     o1, l1, ws1 = binding.decode_device(d, w.softmax_scale, num_splits=4)
     o2, l2, ws2 = binding.decode_device(d, w.softmax_scale, num_splits=4,
-                                        workspace=binding.alloc_workspace(w.B, w.H, 4))
+                                        workspace=binding.alloc_workspace(2, w.H, 4, fp8_max_blocks=w.max_blocks))
     assert binding.mla_get_device_error(ws1) == 0 and binding.mla_get_device_error(ws2) == 0
+    small = binding.alloc_workspace(w.B, w.H, 4)   # split-KV scratch only
+    if binding.mla_decode_fp8_workspace_bytes(1, w.H, w.max_blocks, 1) > small.numel():
+        with pytest.raises(binding.MLAError) as ei:
+            binding.decode_device(d, w.softmax_scale, num_splits=4, workspace=small)
+        assert ei.value.status == 3
     ro, rl = oracle.decode_workload(w)
-    for o, l, what in ((o1, l1, "tensor"), (o2, l2, "cuda-core")):
+    for o, l, what in ((o1, l1, "whole"), (o2, l2, "groups")):
         assert_close(to_np(o).reshape(-1, 512), ro, f"fp8 {what} out")
         assert_close(to_np(l).reshape(-1), rl, f"fp8 {what} lse")
 

@@ -64,6 +64,26 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
 
 
 @pytest.mark.gpu
+def test_noalloc_fp8_beyond_its_room_runs_in_groups():
+    """An fp8 batch whose widened copy (16 sequences x 64 blocks x 72 KB =
+    75 MB) exceeds the 40 MiB array runs in groups of sequences there and
+    matches mla_decode with a whole-batch workspace; the array's error word
+    reads 0 afterwards."""
+    w = inputs.make("fp8", B=16, H=128, L=4096, seed=48)
+    d = binding.to_device(w)
+    assert binding.mla_decode_fp8_workspace_bytes(w.B, w.H, w.max_blocks, 0) > (40 << 20)
+    ref_out, ref_lse, ws = binding.decode_device(d, w.softmax_scale)
+    assert binding.mla_get_device_error(ws) == 0
+    out = torch.full((w.B, w.H, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((w.B, w.H), float("nan"), dtype=torch.float32, device="cuda")
+    st = _noalloc_raw(d, w, out, lse, 0)
+    assert st == 0, binding.STATUS.get(st, st)
+    assert binding.mla_decode_noalloc_get_error() == 0
+    assert_close(to_np(out).reshape(-1, 512), to_np(ref_out).reshape(-1, 512), "noalloc fp8 groups out")
+    assert_close(to_np(lse).reshape(-1), to_np(ref_lse).reshape(-1), "noalloc fp8 groups lse")
+
+
+@pytest.mark.gpu
 def test_noalloc_fp8_cache_matches_decode():
     """An fp8 cache through the built-in scratch: small enough that its
     widened copy fits there, so it takes the tensor-core route as mla_decode
