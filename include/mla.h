@@ -100,7 +100,8 @@ mla_status_t mla_absorb_get_error(void *stream, uint32_t *err_bits);
 
 /*
  * mla_decode_workspace_bytes - bytes of device workspace mla_decode needs for
- * H heads and `num_splits` split-KV partitions (0 = the automatic count the
+ * H heads (mla_decode_multi: H = q_len * heads rows, up to 1024, which above
+ * 128 need the workspace of one 128-row tile) and `num_splits` split-KV partitions (0 = the automatic count the
  * current device would use).  The workspace holds the device error word and
  * the fp32 partial results of sequences that are cut across partitions.
  * Returns 0 on invalid arguments.
@@ -186,7 +187,10 @@ mla_status_t mla_decode(const void *q, mla_cache_dtype_t cache_dtype, const void
  * (the drafts' own rows are already in the cache; causal among the drafts).
  * q: bf16 [B, q_len, H, 576]; out: bf16 [B, q_len, H, 512]; lse: f32
  * [B, q_len, H]; bf16 cache only.  q_len * H must be a multiple of 16 and at
- * most 128.
+ * most 128, or a multiple of 128 up to 1024 with H dividing 128 (e.g. H = 128
+ * and q_len = 2..8): such rows are decoded in tiles of 128 rows (whole
+ * tokens), one kernel pass over the cache per tile, one tile after the other
+ * on `stream`; the tiles read q and write out / lse in place.
  * workspace: mla_decode_workspace_bytes(B, q_len * H, num_splits) bytes.
  * Other arguments and error behaviour as mla_decode; a token that sees no
  * cached token gives out = 0 and lse = -inf.

@@ -2,15 +2,18 @@
 //   q_out[b,h,0:512]   = q_nope[b,h,:] . W_UK[h]      (K = 128, fp32 accumulation, one bf16 rounding)
 //   q_out[b,h,512:576] = q_rope[b,h,:]                (copied)
 //
-// One CTA per (head h, tile of 128 batch rows).  Per head this is a plain GEMM
-// D[128 x 512] = A[128 x 128] . B[128 x 512] with
+// One CTA per (head h, tile of 128 batch rows, half of the 512 columns), two
+// CTAs per SM.  Per head this is a plain GEMM D[128 x 512] = A[128 x 128] .
+// B[128 x 512], each CTA computing one 256-column half:
 //   A = q_nope rows of head h (K-major, rows past B read as zeros by TMA),
-//   B = W_UK[h] stored [d][c] (c contiguous, so MN-major),
-//   D = fp32 in all 512 TMEM columns.
+//   B = the half of W_UK[h] stored [d][c] (c contiguous, so MN-major),
+//   D = fp32 in 256 TMEM columns.
 // The operands are staged by TMA in two K halves (one barrier each) so the
-// MMAs of the first half overlap the second half's load; 16 MMAs of
-// 128 x 256 x 16 in total.  The epilogue: each of the 4 warps reads its 32
-// TMEM lanes (= 32 batch rows) and writes bf16 rows.
+// MMAs of the first half overlap the second half's load; 8 MMAs of
+// 128 x 256 x 16.  The epilogue: each of the 4 warps reads its 32 TMEM lanes
+// (= 32 batch rows) and writes bf16 rows.  Splitting the columns doubles the
+// CTAs of the launch, so that loads, MMAs and stores of the two halves of a
+// head overlap on different SMs instead of running in one CTA in turn.
 #include <cuda.h>
 
 #include <atomic>
@@ -36,9 +39,11 @@ constexpr uint32_t kWBox = 64 * 128;          // [64 d x 64 c] bf16
 constexpr uint32_t kWChunk = 2 * kWBox;       // [128 d x 64 c]: one 64-column chunk of W_UK[h]
 constexpr uint32_t kAOff = 1024;              // after the barrier block
 constexpr uint32_t kWOff = kAOff + 2 * kATile;
-constexpr uint32_t kSmem = kWOff + 8 * kWChunk + 1024;
+constexpr int kCols = 256;                    // columns of D per CTA
+constexpr int kColChunks = kCols / 64;        // 64-column chunks of W_UK per CTA
+constexpr uint32_t kSmem = kWOff + kColChunks * kWChunk + 1024;
 static_assert(kSmem <= 232448, "shared memory budget");
-constexpr uint32_t kHalfBytes = kATile + 8 * kWBox;  // A tile + 8 W boxes per K half
+constexpr uint32_t kHalfBytes = kATile + kColChunks * kWBox;  // A tile + the W boxes per K half
 constexpr uint32_t kIdesc = idesc_bf16(128, 256, false, true);
 
 struct Bars {
@@ -47,7 +52,7 @@ struct Bars {
   uint32_t tmem_base;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 absorb_sm100_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap wmap,
                     const __nv_bfloat16* __restrict__ q_rope, __nv_bfloat16* __restrict__ q_out,
                     int ldq, int B, int H, long long spin_limit) {
@@ -57,6 +62,7 @@ absorb_sm100_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   Bars* bars = reinterpret_cast<Bars*>(smem_raw + (base - raw));
   const int h = blockIdx.x;
   const int b0 = blockIdx.y * 128;
+  const int c0 = blockIdx.z * kCols;            // first output column of this CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ int abort_flag;
 
@@ -68,7 +74,7 @@ absorb_sm100_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_alloc(smem_u32(&bars->tmem_base), kCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -89,9 +95,9 @@ absorb_sm100_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(base + kAOff + kc * kATile),
           "l"(reinterpret_cast<uint64_t>(&qmap)), "r"(64 * kc), "r"(h), "r"(b0), "r"(full)
           : "memory");
-      // W_UK[h] rows d in the same half, all 8 column chunks
-      for (int j = 0; j < 8; ++j)
-        tma_load_2d(base + kWOff + j * kWChunk + kc * kWBox, &wmap, 64 * j, h * 128 + 64 * kc, full);
+      // W_UK[h] rows d in the same half, this CTA's column chunks
+      for (int j = 0; j < kColChunks; ++j)
+        tma_load_2d(base + kWOff + j * kWChunk + kc * kWBox, &wmap, c0 + 64 * j, h * 128 + 64 * kc, full);
     }
     for (int kc = 0; kc < 2; ++kc) {
       if (!wait_phase(smem_u32(&bars->full[kc]), 0, wc)) break;
@@ -100,11 +106,8 @@ absorb_sm100_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       for (int kk = 0; kk < 4; ++kk) {
         const int k = 4 * kc + kk;  // 16-wide step along d
         const uint64_t a = sw128_desc(base + kAOff + kc * kATile + kk * 32, 16, 1024);
-#pragma unroll
-        for (int n = 0; n < 2; ++n) {
-          const uint64_t b = sw128_desc(base + kWOff + 4 * n * kWChunk + k * 2048, kWChunk, 1024);
-          mma_ss(tmem + 256 * n, a, b, kIdesc, k > 0 ? 1u : 0u);
-        }
+        const uint64_t b = sw128_desc(base + kWOff + k * 2048, kWChunk, 1024);
+        mma_ss(tmem, a, b, kIdesc, k > 0 ? 1u : 0u);
       }
     }
     mma_commit(smem_u32(&bars->done));
@@ -118,12 +121,12 @@ absorb_sm100_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   const bool live = ok && b < B;
   __nv_bfloat16* dst = q_out + (size_t(b) * H + h) * ldq;
 #pragma unroll 1
-  for (int ch = 0; ch < 16; ++ch) {
+  for (int ch = 0; ch < kCols / 32; ++ch) {
     uint32_t v[32];
     tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 32 * ch, v);
     tmem_ld_wait();
     if (!live) continue;
-    uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + c0 + 32 * ch);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint32_t w4[4];
@@ -136,7 +139,7 @@ absorb_sm100_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       d4[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
   }
-  if (live && q_rope != nullptr) {
+  if (live && q_rope != nullptr && blockIdx.z == 0) {
     const uint4* src = reinterpret_cast<const uint4*>(q_rope + (size_t(b) * H + h) * kDr);
     uint4* d4 = reinterpret_cast<uint4*>(dst + kDc);
 #pragma unroll
@@ -145,7 +148,7 @@ absorb_sm100_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, 512);
+  if (warp == 0) tmem_dealloc(tmem, kCols);
 }
 
 // ---------------------------------------------------------------- output absorption
@@ -306,7 +309,7 @@ cudaError_t launch_absorb_q(const CUtensorMap& qmap, const CUtensorMap& wmap,
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  dim3 grid(H, (B + 127) / 128);
+  dim3 grid(H, (B + 127) / 128, kDc / kCols);
   absorb_sm100_kernel<<<grid, kThreads, kSmem, stream>>>(qmap, wmap, q_rope, q_out, ldq, B, H,
                                                          spin_limit);
   return cudaGetLastError();

@@ -137,6 +137,15 @@ std::atomic<long long> g_decode_wait_limit{kDefaultSpin};  // set by mla_set_wai
 
 bool valid_heads(int H) { return H >= 16 && H <= kMaxHeads && H % 16 == 0; }
 
+// Multi-token decode with more than 128 query rows per sequence runs in tiles
+// of 128 rows (whole tokens), one decode launch and one cache pass per tile;
+// the tiles read q and write out / lse in place (row stride ld_rows).
+constexpr int kMaxTiledRows = 8 * kMaxHeads;
+
+bool valid_rows(int rows) {
+  return valid_heads(rows) || (rows > kMaxHeads && rows <= kMaxTiledRows && rows % kMaxHeads == 0);
+}
+
 // The fp8 cache's widened bf16 copy, placed after the split-KV workspace:
 // a scratch block table int32 [B * max_blocks] and a dense bf16 cache
 // [B * max_blocks, 64, 576] (block b * max_blocks + j holds logical block j
@@ -180,15 +189,15 @@ long long mla_set_wait_limit(long long cycles) {
 }
 
 size_t mla_decode_workspace_bytes(int B, int H, int num_splits) {
-  if (B < 1 || B > kMaxBatch || !valid_heads(H) || num_splits < 0 || num_splits > kMaxSplits)
+  if (B < 1 || B > kMaxBatch || !valid_rows(H) || num_splits < 0 || num_splits > kMaxSplits)
     return 0;
   int P = resolve_engines(num_splits, B);
   if (P < 1) return 0;
-  return ws_layout(B, H, P).total;
+  return ws_layout(B, H < kMaxHeads ? H : kMaxHeads, P).total;
 }
 
 size_t mla_decode_fp8_workspace_bytes(int B, int H, int max_blocks_per_seq, int num_splits) {
-  if (max_blocks_per_seq < 1 || max_blocks_per_seq > (1 << 24)) return 0;
+  if (max_blocks_per_seq < 1 || max_blocks_per_seq > (1 << 24) || !valid_heads(H)) return 0;
   const size_t base = mla_decode_workspace_bytes(B, H, num_splits);
   if (base == 0) return 0;
   if (static_cast<long long>(B) * max_blocks_per_seq > kMaxWideBlocks) return 0;
@@ -310,8 +319,8 @@ mla_status_t decode_group(DecodeParams p, void* workspace, cudaStream_t st) {
     return fail_with("tensor map encoding failed");
   cudaError_t e = launch_decode_sm100(p, tmap, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = launch_merge_pieces(p.seq_lens, p.B, p.max_blocks, p.H, p.P, p.seq_info, p.lse_part, p.o_part,
-                          p.out, p.lse, p.err, st);
+  e = launch_merge_pieces(p.seq_lens, p.B, p.max_blocks, p.H, p.ld_rows, p.P, p.seq_info, p.lse_part,
+                          p.o_part, p.out, p.lse, p.err, st);
   return status_of(e);
 }
 
@@ -324,9 +333,11 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
                          void* workspace, size_t workspace_bytes, int num_splits, void* stream) {
   if (!q || !cache || !block_table || !seq_lens || !out || !lse || !workspace)
     return MLA_ERR_INVALID_ARG;
-  if (q_len < 1 || q_len > kMaxHeads / 16 || H < 1) return MLA_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > kMaxTiledRows / 16 || H < 1) return MLA_ERR_INVALID_ARG;
   const int rows = H * q_len;
-  if (B < 1 || B > kMaxBatch || !valid_heads(rows)) return MLA_ERR_INVALID_ARG;
+  if (B < 1 || B > kMaxBatch || !valid_rows(rows)) return MLA_ERR_INVALID_ARG;
+  // tiles of 128 rows hold whole tokens: H divides 128
+  if (rows > kMaxHeads && (H % 16 != 0 || kMaxHeads % H != 0)) return MLA_ERR_INVALID_ARG;
   if (q_len > 1 && cache_dtype == MLA_CACHE_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
   if (num_blocks < 1 || max_blocks_per_seq < 1 || max_blocks_per_seq > (1 << 24))
     return MLA_ERR_INVALID_ARG;
@@ -344,7 +355,8 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
     return MLA_ERR_INVALID_ARG;
   const int P = resolve_engines(num_splits, B);
   if (P < 1) return fail_with("no streaming multiprocessor count for the current device");
-  if (workspace_bytes < ws_layout(B, rows, P).total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  const int tile = rows < kMaxHeads ? rows : kMaxHeads;
+  if (workspace_bytes < ws_layout(B, tile, P).total) return MLA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   DecodeParams p;
@@ -353,9 +365,10 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.B = B;
-  p.H = rows;
+  p.H = tile;
   p.q_len = q_len;
   p.h_per_q = H;
+  p.ld_rows = rows;
   p.num_blocks = num_blocks;
   p.max_blocks = max_blocks_per_seq;
   p.softmax_scale = softmax_scale;
@@ -363,7 +376,20 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
   p.lse = lse;
   p.P = P;
   p.spin_limit = g_decode_wait_limit.load();
-  if (!fp8) return decode_group(p, workspace, st);
+  if (!fp8) {
+    // tile t holds rows [128t, 128t + 128): tokens from t0 = 128t / H on,
+    // decoded as the last q_len - t0 tokens of the drafts (so that each row's
+    // causal length comes out right); one launch after the other on `stream`
+    for (int r0 = 0; r0 < rows; r0 += tile) {
+      DecodeParams t = p;
+      t.q = p.q + static_cast<size_t>(r0) * kRow;
+      t.out = p.out + static_cast<size_t>(r0) * kDc;
+      t.lse = p.lse + r0;
+      t.q_len = q_len - r0 / H;
+      if (mla_status_t s = decode_group(t, workspace, st); s != MLA_OK) return s;
+    }
+    return MLA_OK;
+  }
 
   // The fp8 cache: each group of sequences is widened to bf16 rows in the
   // workspace, then decoded like a bf16 cache.  One group when the workspace

@@ -68,7 +68,7 @@ __device__ __forceinline__ void merge_row(int n, LseAt lse_at, OAt o_at, __nv_bf
 
 // grid (B, ceil(H / kRowsPerCta)); warp w merges head blockIdx.y * kRowsPerCta + w.
 __global__ void __launch_bounds__(kMergeThreads)
-merge_pieces_kernel(const int32_t* __restrict__ seq_lens, int max_blocks, int H, int P,
+merge_pieces_kernel(const int32_t* __restrict__ seq_lens, int max_blocks, int H, int ld_rows, int P,
                     const int4* __restrict__ seq_info, const float* __restrict__ lse_part,
                     const float* __restrict__ o_part, __nv_bfloat16* __restrict__ out,
                     float* __restrict__ lse, uint32_t* __restrict__ err) {
@@ -84,12 +84,12 @@ merge_pieces_kernel(const int32_t* __restrict__ seq_lens, int max_blocks, int H,
     L = L < 0 ? 0 : max_blocks * kBlock;
   }
   if (h >= H) return;
-  __nv_bfloat16* row = out + (size_t(b) * H + h) * kDc;
+  __nv_bfloat16* row = out + (size_t(b) * ld_rows + h) * kDc;
   auto fill = [&](float lse_value) {
     uint4* dst = reinterpret_cast<uint4*>(row + lane * 16);
     dst[0] = make_uint4(0u, 0u, 0u, 0u);
     dst[1] = make_uint4(0u, 0u, 0u, 0u);
-    if (lane == 0) lse[size_t(b) * H + h] = lse_value;
+    if (lane == 0) lse[size_t(b) * ld_rows + h] = lse_value;
   };
   if (aborted) {
     fill(NAN);
@@ -113,7 +113,7 @@ merge_pieces_kernel(const int32_t* __restrict__ seq_lens, int max_blocks, int H,
   auto slot_of = [&](int i) { return i == 0 ? slot0 : 2 * (p0 + i); };
   auto lse_at = [&](int i) { return lse_part[size_t(slot_of(i)) * H + h]; };
   auto o_at = [&](int i) { return o_part + (size_t(slot_of(i)) * H + h) * kDc; };
-  merge_row(n, lse_at, o_at, row, lse + size_t(b) * H + h, lane);
+  merge_row(n, lse_at, o_at, row, lse + size_t(b) * ld_rows + h, lane);
 }
 
 // Public combine: o_part [B,H,S,512], lse_part [B,H,S].  grid ceil(B*H / kRowsPerCta).
@@ -129,12 +129,12 @@ combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_p
 
 }  // namespace
 
-cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H, int P,
+cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H, int ld_rows, int P,
                                 const int4* seq_info, const float* lse_part, const float* o_part,
                                 __nv_bfloat16* out, float* lse, uint32_t* err,
                                 cudaStream_t stream) {
   dim3 grid(B, (H + kRowsPerCta - 1) / kRowsPerCta);
-  merge_pieces_kernel<<<grid, kMergeThreads, 0, stream>>>(seq_lens, max_blocks, H, P, seq_info,
+  merge_pieces_kernel<<<grid, kMergeThreads, 0, stream>>>(seq_lens, max_blocks, H, ld_rows, P, seq_info,
                                                           lse_part, o_part, out, lse, err);
   return cudaGetLastError();
 }

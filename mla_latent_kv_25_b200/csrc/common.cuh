@@ -49,7 +49,6 @@ __host__ __device__ inline WsLayout ws_layout(int B, int H, int P) {
 // kind field of seq_info
 constexpr int kSeqWhole = 0;   // one engine wrote out/lse directly
 constexpr int kSeqCut = 1;     // pieces in slots; the merge kernel combines them
-constexpr int kSeqEmpty = 2;   // length 0: out = 0, lse = -inf (written by decode)
 
 // ---------------------------------------------------------------------------
 // Split-KV partition.  The blocks of all sequences are laid end to end

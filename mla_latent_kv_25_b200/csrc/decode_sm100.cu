@@ -316,7 +316,7 @@ __device__ void score_mma(const Ctx& c) {
 __device__ __forceinline__ void load_q_half(const DecodeParams& p, int b, int h, int half, uint32_t taddr,
                                             uint8_t* qrope) {
   const bool live = h < p.H;
-  const uint4* src = reinterpret_cast<const uint4*>(p.q + (size_t(b) * p.H + (live ? h : 0)) * kRow);
+  const uint4* src = reinterpret_cast<const uint4*>(p.q + (size_t(b) * p.ld_rows + (live ? h : 0)) * kRow);
   const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
   for (int pair = 0; pair < 2; ++pair) {
@@ -347,7 +347,7 @@ __device__ __forceinline__ void load_q_half(const DecodeParams& p, int b, int h,
 
 __device__ __forceinline__ void prefetch_q_row_l2(const DecodeParams& p, int b, int h) {
   if (h >= p.H) return;
-  const char* src = reinterpret_cast<const char*>(p.q + (size_t(b) * p.H + h) * kRow);
+  const char* src = reinterpret_cast<const char*>(p.q + (size_t(b) * p.ld_rows + h) * kRow);
 #pragma unroll
   for (int i = 0; i < 9; ++i) asm volatile("prefetch.global.L2 [%0];" ::"l"(src + 128 * i));
 }
@@ -794,7 +794,7 @@ __device__ void value_epilogue(const Ctx& c) {
         if (!live) continue;
         const int col = ocol + 32 * ch;
         if (g.slot < 0) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t(g.b) * p.H + h) * kDc + col);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t(g.b) * p.ld_rows + h) * kDc + col);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t w4[4];
@@ -818,7 +818,7 @@ __device__ void value_epilogue(const Ctx& c) {
       mbar_arrive(bar_addr(c.bars->o_free));
       if (live && half == 0) {
         if (g.slot < 0)
-          p.lse[size_t(g.b) * p.H + h] = lse;
+          p.lse[size_t(g.b) * p.ld_rows + h] = lse;
         else
           p.lse_part[size_t(g.slot) * p.H + h] = lse;
       }

@@ -27,6 +27,9 @@ struct DecodeParams {
   // h_per_q heads each (row r = token r / h_per_q); token j sees the
   // sequence without its last q_len - 1 - j tokens.  q_len = 1: plain decode.
   int q_len, h_per_q;
+  // Rows between consecutive sequences in q, out and lse (= H, or the whole
+  // q_len * heads of a sequence when its rows are decoded in tiles of 128).
+  int ld_rows;
 };
 
 // Tensor-core decode (bf16 cache): clusters of two CTAs, one engine each.
@@ -36,7 +39,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, 
 size_t decode_sm100_smem_bytes();
 int decode_sm100_max_clusters();
 
-cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H, int P,
+cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, int H, int ld_rows, int P,
                                 const int4* seq_info, const float* lse_part, const float* o_part,
                                 __nv_bfloat16* out, float* lse, uint32_t* err,
                                 cudaStream_t stream);

@@ -66,7 +66,12 @@ def test_workspace_size_and_validation_without_device():
     # room for 2 fp32 pieces (512 + lse) per engine and head
     assert n1 >= 2 * 74 * 128 * 513 * 4
     assert lib.mla_decode_workspace_bytes(64, 100, 74) == 0     # H not a multiple of 16
-    assert lib.mla_decode_workspace_bytes(64, 256, 74) == 0     # H > 128
+    # multi-token rows above 128 run in 128-row tiles: the workspace of one tile
+    assert lib.mla_decode_workspace_bytes(64, 256, 74) == n1
+    assert lib.mla_decode_workspace_bytes(64, 1024, 74) == n1
+    assert lib.mla_decode_workspace_bytes(64, 192, 74) == 0     # not whole 128-row tiles
+    assert lib.mla_decode_workspace_bytes(64, 1152, 74) == 0    # more than 8 tiles
+    assert lib.mla_decode_fp8_workspace_bytes(64, 256, 4, 74) == 0  # fp8: one token per sequence
     assert lib.mla_decode_workspace_bytes(0, 128, 74) == 0
     assert lib.mla_decode_workspace_bytes(1, 128, -1) == 0
 
@@ -165,7 +170,8 @@ def test_absorb_and_combine_reject_invalid_arguments_on_host():
     # multi-token decode: q_len * H must be a multiple of 16 and at most 128
     assert lib.mla_decode_multi(g, 0, g, g, g, 1, 16, 1, 1, 0.1, g, g, g, 1 << 20, 0, None) == 1
     assert lib.mla_decode_multi(g, 3, g, g, g, 1, 8, 1, 1, 0.1, g, g, g, 1 << 20, 0, None) == 1
-    assert lib.mla_decode_multi(g, 2, g, g, g, 1, 128, 1, 1, 0.1, g, g, g, 1 << 20, 0, None) == 1
+    assert lib.mla_decode_multi(g, 2, g, g, g, 1, 96, 1, 1, 0.1, g, g, g, 1 << 20, 0, None) == 1  # 192 rows: not whole 128-row tiles
+    assert lib.mla_decode_multi(g, 3, g, g, g, 1, 128, 1, 1, 0.1, g, g, g, 1 << 20, 9, None) == 3  # tiles need one 128-row workspace
     assert lib.mla_decode_multi(None, 2, g, g, g, 1, 16, 1, 1, 0.1, g, g, g, 1 << 20, 0, None) == 1
     assert lib.mla_combine(None, g, 1, 16, 2, g, g, None) == 1
     assert lib.mla_combine(g, g, 1, 16, 0, g, g, None) == 1

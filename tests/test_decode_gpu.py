@@ -255,11 +255,14 @@ def _multi_reference(w, q_len, H):
                                units=oracle.all_units(B * q_len, H), cache_kind=w.cache_dtype)
 
 
-@pytest.mark.parametrize("q_len,H,num_splits", [(2, 32, 0), (2, 64, 5), (4, 32, 3), (4, 16, 0)])
+@pytest.mark.parametrize("q_len,H,num_splits", [(2, 32, 0), (2, 64, 5), (4, 32, 3), (4, 16, 0),
+                                               (2, 128, 0), (4, 128, 5), (4, 64, 4)])
 def test_multi_token_decode_matches_oracle(q_len, H, num_splits):
     """q_len query tokens per sequence share the cache pass; token j is causal
     among the drafts (sees all but the last q_len - 1 - j tokens).  Lengths
-    include one shorter than q_len (its first tokens see nothing)."""
+    include one shorter than q_len (its first tokens see nothing).  Above 128
+    rows (H = 128 with 2 and 4 tokens, 4 x 64) the rows run in
+    tiles of 128, one cache pass each."""
     B = 4
     w = inputs.make("v3", B=B, H=q_len * H, L=[700, 65, 130, 2], seed=46, q_std=2.0)
     d = binding.to_device(w)
@@ -277,33 +280,20 @@ def test_multi_token_decode_matches_oracle(q_len, H, num_splits):
     assert_close(to_np(lse).reshape(-1)[finite], rl[finite], f"multi lse q_len={q_len}")
 
 
-# ---------------------------------------------------------------- full-size configs, sampled rows
-
-def _sample_rows(w, n, seed):
-    rng = np.random.default_rng(seed)
-    nz = np.nonzero(w.seq_lens.numpy() > 0)[0]
-    b = rng.choice(nz, size=n, replace=True)
-    h = rng.integers(0, w.H, size=n)
-    rows = np.unique(np.stack([b, h], 1), axis=0)
-    # always include the longest sequence's first and last head
-    bl = int(np.argmax(w.seq_lens.numpy()))
-    return np.concatenate([rows, [[bl, 0], [bl, w.H - 1]]]).astype(np.int32)
-
+# ---------------------------------------------------------------- full-size configs, every row
 
 @pytest.mark.parametrize("name", ["v3", "ragged", "long", "fp8"])
-def test_full_config_sampled_rows(name):
+def test_full_config_every_row(name):
+    """Every output row and lse of each full-size workload, in the launch
+    configuration the benchmark times (automatic split count), against the
+    oracle computed for the whole workload (multithreaded fp64 C: a few
+    seconds to tens of seconds per workload on the host cores)."""
     w = inputs.make(name)
     out, lse, err = run(w)
     assert err == 0
-    rows = _sample_rows(w, 48 if name != "long" else 24, seed=1)
-    ro, rl = oracle.decode_workload(w, rows=rows)
-    o = to_np(out)[rows[:, 0], rows[:, 1]]
-    l = to_np(lse)[rows[:, 0], rows[:, 1]]
-    assert_close(o, ro, name + " out")
-    assert_close(l, rl, name + " lse")
-    # properties at full size: every row finite, lse >= max-free lower bound log(1)
-    assert np.all(np.isfinite(to_np(out)))
-    assert np.all(np.isfinite(to_np(lse)))
+    ro, rl = oracle.decode_workload(w)
+    assert_close(to_np(out).reshape(-1, 512), ro, name + " out")
+    assert_close(to_np(lse).reshape(-1), rl, name + " lse")
 
 
 # ---------------------------------------------------------------- determinism under load
