@@ -314,10 +314,16 @@ mla_status_t decode_group(DecodeParams p, void* workspace, cudaStream_t st) {
   p.seq_info = reinterpret_cast<int4*>(wsb + ws.seq_info);
   p.lse_part = reinterpret_cast<float*>(wsb + ws.lse_part);
   p.o_part = reinterpret_cast<float*>(wsb + ws.o_part);
-  CUtensorMap tmap;
+  CUtensorMap tmap, qmap;
   if (!encode_bf16_map(&tmap, p.cache, uint64_t(p.num_blocks) * kBlock, kRow, kRow * 2))
     return fail_with("tensor map encoding failed");
-  cudaError_t e = launch_decode_sm100(p, tmap, st);
+  {
+    cuuint64_t dims[2] = {uint64_t(kRow), uint64_t(p.B - 1) * uint64_t(p.ld_rows) + uint64_t(p.H)};
+    cuuint64_t strides[1] = {uint64_t(kRow) * 2};
+    cuuint32_t box[2] = {64, 128};
+    if (!encode_bf16(&qmap, p.q, 2, dims, strides, box)) return fail_with("query tensor map encoding failed");
+  }
+  cudaError_t e = launch_decode_sm100(p, tmap, qmap, st);
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch_merge_pieces(p.seq_lens, p.B, p.max_blocks, p.H, p.ld_rows, p.P, p.seq_info, p.lse_part,
                           p.o_part, p.out, p.lse, p.err, st);

@@ -72,6 +72,9 @@ merge_pieces_kernel(const int32_t* __restrict__ seq_lens, int max_blocks, int H,
                     const int4* __restrict__ seq_info, const float* __restrict__ lse_part,
                     const float* __restrict__ o_part, __nv_bfloat16* __restrict__ out,
                     float* __restrict__ lse, uint32_t* __restrict__ err) {
+  // launched with programmatic stream serialization right behind the decode:
+  // wait for it to complete (and its writes to be visible) before any read
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31;
   const int h = blockIdx.y * kRowsPerCta + (threadIdx.x >> 5);
@@ -133,10 +136,17 @@ cudaError_t launch_merge_pieces(const int32_t* seq_lens, int B, int max_blocks, 
                                 const int4* seq_info, const float* lse_part, const float* o_part,
                                 __nv_bfloat16* out, float* lse, uint32_t* err,
                                 cudaStream_t stream) {
-  dim3 grid(B, (H + kRowsPerCta - 1) / kRowsPerCta);
-  merge_pieces_kernel<<<grid, kMergeThreads, 0, stream>>>(seq_lens, max_blocks, H, ld_rows, P, seq_info,
-                                                          lse_part, o_part, out, lse, err);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B, (H + kRowsPerCta - 1) / kRowsPerCta);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_pieces_kernel, seq_lens, max_blocks, H, ld_rows, P, seq_info,
+                            lse_part, o_part, out, lse, err);
 }
 
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int B, int H, int S,

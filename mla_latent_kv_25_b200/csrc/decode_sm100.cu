@@ -90,6 +90,7 @@ struct Barriers {
   uint64_t k_full[kKSlots], k_empty[kKSlots];
   uint64_t s_full, s_empty;
   uint64_t q_ready, q_free;
+  uint64_t q_full, qstage_free;      // first segment: query tile staged by TMA
   uint64_t xchg[4];                 // softmax: the two threads of a head swap max / sum
   uint64_t p_empty[kNP];            // score CTA: record r of the value CTA is free
   uint64_t v_full[kVSlots], v_empty[kVSlots], v_fixed[kVSlots];
@@ -109,6 +110,11 @@ constexpr uint32_t kXchgBytes = 2 * 2 * 128 * 4;
 constexpr uint32_t kQRopeOff = kRegion + 3072;               // 1024-aligned
 __host__ __device__ constexpr uint32_t k_slot_off(int s) { return kQRopeOff + kQTile + s * kKSlot; }
 constexpr uint32_t kScoreSmem = k_slot_off(kKSlots);
+// the first segment's query [128 rows x 512] lands by TMA in K slots 1-2
+// (eight 16 KB column chunks, 128 B swizzle) before those slots' first fill;
+// its RoPE columns land straight in the RoPE tile
+constexpr uint32_t kQStageOff = k_slot_off(1);
+static_assert(kKSlots >= 3 && 2 * kKSlot >= 8 * kQTile, "query staging room");
 // value CTA: V ring, P records
 __host__ __device__ constexpr uint32_t v_slot_off(int s) { return kRegion + s * kVSlot; }
 __host__ __device__ constexpr uint32_t rec_off(int r) { return kRegion + kVSlots * kVSlot + r * kRecBytes; }
@@ -176,7 +182,7 @@ __device__ __forceinline__ int block_rows(const DecodeParams& p, const Segment& 
 // Four consecutive blocks of a segment form one pass (fewer at the end of the
 // segment); each pass streams its 9 column chunks through the slot ring, two
 // chunks of all the pass's blocks per slot (the RoPE chunk alone).
-__device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
+__device__ void score_tma(const Ctx& c, const CUtensorMap* tmap, const CUtensorMap* qmap) {
   const DecodeParams& p = *c.p;
   SegWalker w;
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
@@ -184,9 +190,23 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
   BlockCursor cur;
   uint32_t fit = 0;
   bool alive = true;
-  if (c.lane == 0) prefetch_tmap(tmap);
+  bool first = true;
+  if (c.lane == 0) {
+    prefetch_tmap(tmap);
+    prefetch_tmap(qmap);
+  }
   while (alive && w.next(g)) {
     cur.reset(p, g);
+    if (first && c.lane == 0) {
+      // the engine's first query tile: eight latent chunks into K slots 1-2,
+      // the RoPE chunk into its tile
+      const uint32_t full = bar_addr(c.bars->q_full);
+      mbar_arrive_expect_tx(full, 9 * kQTile);
+      const int row = g.b * p.ld_rows;
+      for (int ch = 0; ch < 8; ++ch) tma_load_2d(c.base + kQStageOff + ch * kQTile, qmap, 64 * ch, row, full);
+      tma_load_2d(c.base + kQRopeOff, qmap, kDc, row, full);
+    }
+    first = false;
     for (int j = g.blk_lo; alive && j < g.blk_hi; j += kPassBlocks) {
       const int nb = min(kPassBlocks, g.blk_hi - j);
       int blk[kPassBlocks];
@@ -202,6 +222,11 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap) {
       for (int f = 0; f < kFills; ++f, ++fit) {
         const int s = fit % kKSlots;
         if (!warp_wait(bar_addr(c.bars->k_empty[s]), ((fit / kKSlots) & 1u) ^ 1u, c.wc)) {
+          alive = false;
+          break;
+        }
+        // slots 1-2 hold the first query tile until the softmax warps took it
+        if (fit == 1 && !warp_wait(bar_addr(c.bars->qstage_free), 0, c.wc)) {
           alive = false;
           break;
         }
@@ -345,6 +370,35 @@ __device__ __forceinline__ void load_q_half(const DecodeParams& p, int b, int h,
   }
 }
 
+// The first segment's query row h from the TMA-staged tile: half 0 moves
+// chunks 0-3 into TMEM lane h, half 1 chunks 4-7; rows at or past H (padding
+// heads) get zeros, also in the RoPE tile the TMA filled.
+__device__ __forceinline__ void q_half_from_stage(const Ctx& c, int h, int half, int H, uint32_t taddr,
+                                                  uint8_t* qrope) {
+  const bool live = h < H;
+  const uint32_t swz = static_cast<uint32_t>(h & 7);
+  const uint8_t* stage = c.gbase + kQStageOff + h * 128;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int ch = 4 * half + k;
+    uint32_t r[32];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const uint4 u = live ? *reinterpret_cast<const uint4*>(stage + ch * kQTile + ((static_cast<uint32_t>(v) ^ swz) << 4))
+                           : make_uint4(0, 0, 0, 0);
+      r[4 * v] = u.x;
+      r[4 * v + 1] = u.y;
+      r[4 * v + 2] = u.z;
+      r[4 * v + 3] = u.w;
+    }
+    tmem_st32(taddr + kQCol + 32 * ch, r);
+  }
+  if (half == 1 && !live) {
+#pragma unroll
+    for (int v = 0; v < 8; ++v) *reinterpret_cast<uint4*>(qrope + h * 128 + v * 16) = make_uint4(0, 0, 0, 0);
+  }
+}
+
 __device__ __forceinline__ void prefetch_q_row_l2(const DecodeParams& p, int b, int h) {
   if (h >= p.H) return;
   const char* src = reinterpret_cast<const char*>(p.q + (size_t(b) * p.ld_rows + h) * kRow);
@@ -391,7 +445,14 @@ __device__ void score_softmax(const Ctx& c) {
       if (!warp_wait(bar_addr(c.bars->q_free), (seg - 1) & 1u, c.wc)) break;
       tc_fence_after();
     }
-    load_q_half(p, g.b, h, half, c.tmem + lane_off, qrope);
+    if (seg == 0) {
+      if (!warp_wait(bar_addr(c.bars->q_full), 0, c.wc)) break;
+      q_half_from_stage(c, h, half, p.H, c.tmem + lane_off, qrope);
+      __syncwarp();
+      if (c.lane == 0) mbar_arrive(bar_addr(c.bars->qstage_free));
+    } else {
+      load_q_half(p, g.b, h, half, c.tmem + lane_off, qrope);
+    }
     fence_proxy_async_smem();
     tmem_st_wait();
     tc_fence_before();
@@ -831,7 +892,8 @@ __device__ void value_epilogue(const Ctx& c) {
 // ============================================================ kernel
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p) {
+decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap qmap,
+                    const DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -850,6 +912,8 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
     mbar_init(smem_u32(&bars->s_empty), 256);       // every softmax thread
     mbar_init(smem_u32(&bars->q_ready), 256);
     mbar_init(smem_u32(&bars->q_free), 1);
+    mbar_init(smem_u32(&bars->q_full), 1);
+    mbar_init(smem_u32(&bars->qstage_free), 8);     // lane 0 of every softmax warp
     for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&bars->xchg[q]), 64);  // two warps
     for (int r = 0; r < kNP; ++r) {
       mbar_init(smem_u32(&bars->p_empty[r]), 1);      // PV commit, or the epilogue (segment end)
@@ -874,6 +938,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
+  // launched with programmatic stream serialization: the set-up above ran
+  // while the previous kernel on the stream finished; every global read and
+  // write comes after this wait.  The merge kernel that follows may be
+  // scheduled now (it waits for this grid to complete before its work).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   Ctx c;
   c.p = &p;
@@ -888,7 +958,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
 
   if (warp < 4) {
     if (rank == 0) {
-      if (warp == 0) score_tma(c, &tmap);
+      if (warp == 0) score_tma(c, &tmap, &qmap);
       else if (warp == 1) score_mma(c);
     } else {
       if (warp == 0) value_tma(c, &tmap);
@@ -920,7 +990,8 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams
 
 size_t decode_sm100_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, cudaStream_t stream) {
+cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, const CUtensorMap& qmap,
+                                cudaStream_t stream) {
   static bool attr_set[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
@@ -931,8 +1002,17 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, 
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  decode_sm100_kernel<<<dim3(2 * p.P), kThreads, kSmemBytes, stream>>>(tmap, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * p.P);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_sm100_kernel, tmap, qmap, p);
 }
 
 int decode_sm100_max_clusters() {

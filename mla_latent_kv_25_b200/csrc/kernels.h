@@ -35,7 +35,10 @@ struct DecodeParams {
 // Tensor-core decode (bf16 cache): clusters of two CTAs, one engine each.
 // `tmap` is a 2-D tiled map over the cache viewed as [num_blocks*64, 576]
 // bf16 with a 64 x 64 box and 128-byte swizzle.
-cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, cudaStream_t stream);
+// `qmap`: 2-D map over q viewed as [(B - 1) * ld_rows + H, 576] bf16, 64 x 128
+// box, 128-byte swizzle (the first query tile of every engine).
+cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, const CUtensorMap& qmap,
+                                cudaStream_t stream);
 size_t decode_sm100_smem_bytes();
 int decode_sm100_max_clusters();
 

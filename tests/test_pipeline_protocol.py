@@ -62,6 +62,7 @@ def roles(segs, rescale, k_slots, n_rec):
         bar(f"k_full{i}", 1); bar(f"k_empty{i}", 1)
     bar("s_full", 1); bar("s_empty", 256)
     bar("q_ready", 256); bar("q_free", 1)
+    bar("q_full", 1); bar("qstage_free", 8)          # first query tile staged in K slots 1-2
     bar("xchg", 2)                                   # one quadrant's two warps, one per half
     for i in range(n_rec):
         bar(f"p_full{i}", 4)                         # the four warps of the writing half
@@ -75,11 +76,15 @@ def roles(segs, rescale, k_slots, n_rec):
 
     def score_tma():
         fit = 0
-        for lo, hi in segs:
+        for seg, (lo, hi) in enumerate(segs):
+            if seg == 0:
+                B["q_full"].arrive()                 # the first query tile's bytes land
             for _j, _nb in _passes(lo, hi):
                 for _f in range(FILLS):
                     s = fit % k_slots
                     yield wait(f"k_empty{s}", ((fit // k_slots) & 1) ^ 1, fit // k_slots - 1)
+                    if fit == 1:                     # slots 1-2 free once the tile moved to TMEM
+                        yield wait("qstage_free", 0, 0)
                     B[f"k_full{s}"].arrive()
                     fit += 1
 
@@ -103,6 +108,9 @@ def roles(segs, rescale, k_slots, n_rec):
         for seg, (lo, hi) in enumerate(segs):
             if seg > 0:
                 yield wait("q_free", (seg - 1) & 1, seg - 1)
+            else:
+                yield wait("q_full", 0, 0)
+                B["qstage_free"].arrive(4)           # lane 0 of each of the half's four warps
             B["q_ready"].arrive(128)
             for j0, nb in _passes(lo, hi):
                 yield wait("s_full", pit & 1, pit)
