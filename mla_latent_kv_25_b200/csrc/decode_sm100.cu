@@ -29,9 +29,11 @@
 // with A in TMEM, the PV at ~129); an mbarrier probe between MMAs stalls the
 // issue stream unless it is issued ahead of the MMAs it guards, so every MMA
 // loop polls the next stage's barrier before issuing the current stage; the
-// SM-to-SM hand-off peaks at ~21 bytes per clock, and only for whole 32-byte
-// sectors: a lane's 16-byte store alone moves half as much, so lanes pair up
-// to write both halves of a sector.
+// SM-to-SM hand-off peaks at ~21 bytes per clock, and only when the stores
+// of a warp fill whole 128-byte lines (16-byte stores to 32 different lines,
+// or 32-byte sectors of them, move half as much), so P crosses without
+// swizzle, in 8 x 8 core matrices: chunk c of 32 heads is 512 contiguous
+// bytes.
 //
 // Heads are the M = 128 dimension of both contractions (padded with zero query
 // rows for H < 128).  The running max of a head moves only when a pass's max
@@ -70,6 +72,7 @@ constexpr uint32_t kPassChunk = kPassBlocks * kChunk;  // one column chunk of a 
 constexpr uint32_t kKSlot = 2 * kPassChunk;     // two column chunks of a pass
 constexpr uint32_t kVSlot = 4 * kChunk;         // [64 rows x 256 bf16]
 constexpr uint32_t kPBytes = 128 * 64 * 2;      // P [128 heads x 64 tokens] bf16
+constexpr uint32_t kPCoreK = 128 * 16;          // P: bytes per 8-token column of core matrices
 constexpr uint32_t kMetaBytes = 128 * 16;       // per head: alpha, m, l, unused
 constexpr uint32_t kFlagBytes = 64;             // per quadrant: rescale flag
 constexpr uint32_t kRecBytes = 19 * 1024;       // one record (P, meta, flags), 1 KB aligned
@@ -566,11 +569,9 @@ __device__ void score_softmax(const Ctx& c) {
         const bool meta = kb == 0 || (last_pass && kb == nb - 1);
         if (c.lane == 0) mbar_arrive_expect_tx_cluster_relaxed(full, 32 * (128 + (meta ? 16 : 0)) + 4);
         float sum0 = 0.f, sum1 = 0.f;
-        // chunks 2t and 2t+1 of a row share a 32-byte sector of the record;
-        // lanes 2i and 2i+1 trade one chunk each so that every store writes
-        // a whole sector (row 2i, then row 2i+1)
-        const bool odd = c.lane & 1;
-        const uint32_t row_a = static_cast<uint32_t>(h & ~1), row_b = row_a + 1;
+        // the record holds P without swizzle in 8 x 8 core matrices (token
+        // chunk c of heads 8i..8i+7 in 128 contiguous bytes): the 32 lanes'
+        // 16-byte chunks c of one warp fill four whole 128-byte lines
 #pragma unroll
         for (int tp = 0; tp < 4; ++tp) {
           uint32_t pk[2][4];
@@ -586,16 +587,10 @@ __device__ void score_softmax(const Ctx& c) {
               __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
               pk[u][e] = *reinterpret_cast<uint32_t*>(&b2);
             }
-          uint32_t d1[4], d2[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t got = __shfl_xor_sync(0xffffffffu, odd ? pk[0][e] : pk[1][e], 1);
-            d1[e] = odd ? got : pk[0][e];   // row 2i: chunk 2t (even lane), 2t+1 (odd lane)
-            d2[e] = odd ? pk[1][e] : got;   // row 2i+1: chunk 2t (even lane), 2t+1 (odd lane)
-          }
-          const uint32_t chl = static_cast<uint32_t>(2 * tp) | (odd ? 1u : 0u);
-          st_async_v4(rec + row_a * 128 + ((chl ^ (row_a & 7)) << 4), make_uint4(d1[0], d1[1], d1[2], d1[3]), full);
-          st_async_v4(rec + row_b * 128 + ((chl ^ (row_b & 7)) << 4), make_uint4(d2[0], d2[1], d2[2], d2[3]), full);
+          for (int u = 0; u < 2; ++u)
+            st_async_v4(rec + (2 * tp + u) * kPCoreK + h * 16, make_uint4(pk[u][0], pk[u][1], pk[u][2], pk[u][3]),
+                        full);
         }
         l += sum0 + sum1;
         if (c.lane == 0) st_async_b32(rec + kPBytes + kMetaBytes + q4 * 4, (kb == 0 && any) ? 1u : 0u, full);
@@ -770,7 +765,7 @@ __device__ bool value_mma_segment(const Ctx& c, const Segment& g, uint32_t seg, 
       const uint32_t va = c.base + v_slot_off(s);
 #pragma unroll
       for (int k = 0; k < kBlock / 16; ++k)
-        mma_ss(c.tmem + 256 * n, sw128_desc(pa + k * 32, 16, 1024),
+        mma_ss(c.tmem + 256 * n, plain_desc(pa + k * 2 * kPCoreK, kPCoreK, 128),
                sw128_desc(va + k * 2048, kChunk, 1024), kIdescPV, (k > 0 || !first) ? 1u : 0u);
       mma_commit(bar_addr(c.bars->v_empty[s]));
     }

@@ -410,6 +410,18 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// Shared-memory matrix descriptor without swizzle: 8 x 16-byte core matrices
+// of 128 contiguous bytes; for a K-major operand `lbo` is the byte stride
+// between core matrices along K and `sbo` the stride between 8-row groups.
+__device__ __forceinline__ uint64_t plain_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100; swizzle mode 0: none
+  return d;
+}
+
 // Instruction descriptor: kind::f16 with bf16 A/B, fp32 D; M x N; operand majors.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                   // D format f32
