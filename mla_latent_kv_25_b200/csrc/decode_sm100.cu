@@ -93,7 +93,7 @@ struct Barriers {
   uint64_t k_full[kKSlots], k_empty[kKSlots];
   uint64_t s_full, s_empty;
   uint64_t q_ready, q_free;
-  uint64_t q_full, qstage_free;      // first segment: query tile staged by TMA
+  uint64_t q_full, qstage_free;      // a segment's query tile staged by TMA
   uint64_t xchg[4];                 // softmax: the two threads of a head swap max / sum
   uint64_t p_empty[kNP];            // score CTA: record r of the value CTA is free
   uint64_t v_full[kVSlots], v_empty[kVSlots], v_fixed[kVSlots];
@@ -113,9 +113,9 @@ constexpr uint32_t kXchgBytes = 2 * 2 * 128 * 4;
 constexpr uint32_t kQRopeOff = kRegion + 3072;               // 1024-aligned
 __host__ __device__ constexpr uint32_t k_slot_off(int s) { return kQRopeOff + kQTile + s * kKSlot; }
 constexpr uint32_t kScoreSmem = k_slot_off(kKSlots);
-// the first segment's query [128 rows x 512] lands by TMA in K slots 1-2
-// (eight 16 KB column chunks, 128 B swizzle) before those slots' first fill;
-// its RoPE columns land straight in the RoPE tile
+// each segment's query [128 rows x 512] lands by TMA in K slots 1-2 (eight
+// 16 KB column chunks, 128 B swizzle) while the ring is empty, before those
+// slots' next fill; its RoPE columns land straight in the RoPE tile
 constexpr uint32_t kQStageOff = k_slot_off(1);
 static_assert(kKSlots >= 3 && 2 * kKSlot >= 8 * kQTile, "query staging room");
 // value CTA: V ring, P records
@@ -191,25 +191,34 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap, const CUtensorM
   w.init(p.seq_lens, p.B, p.max_blocks, p.P, c.engine);
   Segment g;
   BlockCursor cur;
-  uint32_t fit = 0;
+  uint32_t fit = 0, seg = 0;
   bool alive = true;
-  bool first = true;
   if (c.lane == 0) {
     prefetch_tmap(tmap);
     prefetch_tmap(qmap);
   }
   while (alive && w.next(g)) {
     cur.reset(p, g);
-    if (first && c.lane == 0) {
-      // the engine's first query tile: eight latent chunks into K slots 1-2,
-      // the RoPE chunk into its tile
+    // the segment's query tile goes to K slots 1-2 (eight latent chunks) and
+    // the RoPE tile: after the previous segment's last fill has been consumed
+    // (the MMAs take fills in order, so the whole ring is then free and the
+    // RoPE tile no longer read)
+    if (fit > 0) {
+      const uint32_t k = fit - 1;
+      if (!warp_wait(bar_addr(c.bars->k_empty[k % kKSlots]), (k / kKSlots) & 1u, c.wc)) {
+        alive = false;
+        break;
+      }
+    }
+    if (c.lane == 0) {
       const uint32_t full = bar_addr(c.bars->q_full);
       mbar_arrive_expect_tx(full, 9 * kQTile);
       const int row = g.b * p.ld_rows;
       for (int ch = 0; ch < 8; ++ch) tma_load_2d(c.base + kQStageOff + ch * kQTile, qmap, 64 * ch, row, full);
       tma_load_2d(c.base + kQRopeOff, qmap, kDc, row, full);
     }
-    first = false;
+    __syncwarp();
+    bool staged = true;  // slots 1-2 hold the query until the softmax warps took it
     for (int j = g.blk_lo; alive && j < g.blk_hi; j += kPassBlocks) {
       const int nb = min(kPassBlocks, g.blk_hi - j);
       int blk[kPassBlocks];
@@ -228,10 +237,12 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap, const CUtensorM
           alive = false;
           break;
         }
-        // slots 1-2 hold the first query tile until the softmax warps took it
-        if (fit == 1 && !warp_wait(bar_addr(c.bars->qstage_free), 0, c.wc)) {
-          alive = false;
-          break;
+        if (staged && s != 0) {
+          if (!warp_wait(bar_addr(c.bars->qstage_free), seg & 1u, c.wc)) {
+            alive = false;
+            break;
+          }
+          staged = false;
         }
         if (c.lane == 0) {
           const int nch = f < 4 ? 2 : 1;
@@ -247,6 +258,7 @@ __device__ void score_tma(const Ctx& c, const CUtensorMap* tmap, const CUtensorM
         __syncwarp();
       }
     }
+    ++seg;
   }
   // wait (bounded) for the loads this warp issued before the CTA may exit
   if (!alive) {
@@ -337,43 +349,7 @@ __device__ void score_mma(const Ctx& c) {
   }
 }
 
-// Query row of sequence b for head h, one half per thread: half 0 writes
-// columns 0..255 into TMEM lane h (Q chunks 0-3), half 1 columns 256..511
-// (chunks 4-7) and the RoPE columns 512..575 into the swizzled shared-memory
-// tile (row h).  All global loads of a thread are issued before any store.
-__device__ __forceinline__ void load_q_half(const DecodeParams& p, int b, int h, int half, uint32_t taddr,
-                                            uint8_t* qrope) {
-  const bool live = h < p.H;
-  const uint4* src = reinterpret_cast<const uint4*>(p.q + (size_t(b) * p.ld_rows + (live ? h : 0)) * kRow);
-  const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-  for (int pair = 0; pair < 2; ++pair) {
-    uint4 v8[16];
-#pragma unroll
-    for (int v = 0; v < 16; ++v) v8[v] = live ? __ldg(src + (4 * half + 2 * pair) * 8 + v) : z;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      uint32_t r[32];
-#pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        r[4 * v] = v8[8 * hh + v].x;
-        r[4 * v + 1] = v8[8 * hh + v].y;
-        r[4 * v + 2] = v8[8 * hh + v].z;
-        r[4 * v + 3] = v8[8 * hh + v].w;
-      }
-      tmem_st32(taddr + kQCol + 32 * (4 * half + 2 * pair + hh), r);
-    }
-  }
-  if (half == 1) {
-    const uint32_t swz = static_cast<uint32_t>(h & 7);
-    uint8_t* row = qrope + h * 128;
-#pragma unroll
-    for (int v = 0; v < 8; ++v)
-      *reinterpret_cast<uint4*>(row + ((static_cast<uint32_t>(v) ^ swz) << 4)) = live ? __ldg(src + 64 + v) : z;
-  }
-}
-
-// The first segment's query row h from the TMA-staged tile: half 0 moves
+// A segment's query row h from the TMA-staged tile: half 0 moves
 // chunks 0-3 into TMEM lane h, half 1 chunks 4-7; rows at or past H (padding
 // heads) get zeros, also in the RoPE tile the TMA filled.
 __device__ __forceinline__ void q_half_from_stage(const Ctx& c, int h, int half, int H, uint32_t taddr,
@@ -448,14 +424,10 @@ __device__ void score_softmax(const Ctx& c) {
       if (!warp_wait(bar_addr(c.bars->q_free), (seg - 1) & 1u, c.wc)) break;
       tc_fence_after();
     }
-    if (seg == 0) {
-      if (!warp_wait(bar_addr(c.bars->q_full), 0, c.wc)) break;
-      q_half_from_stage(c, h, half, p.H, c.tmem + lane_off, qrope);
-      __syncwarp();
-      if (c.lane == 0) mbar_arrive(bar_addr(c.bars->qstage_free));
-    } else {
-      load_q_half(p, g.b, h, half, c.tmem + lane_off, qrope);
-    }
+    if (!warp_wait(bar_addr(c.bars->q_full), seg & 1u, c.wc)) break;
+    q_half_from_stage(c, h, half, p.H, c.tmem + lane_off, qrope);
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(bar_addr(c.bars->qstage_free));
     fence_proxy_async_smem();
     tmem_st_wait();
     tc_fence_before();

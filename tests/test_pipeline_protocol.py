@@ -62,7 +62,7 @@ def roles(segs, rescale, k_slots, n_rec):
         bar(f"k_full{i}", 1); bar(f"k_empty{i}", 1)
     bar("s_full", 1); bar("s_empty", 256)
     bar("q_ready", 256); bar("q_free", 1)
-    bar("q_full", 1); bar("qstage_free", 8)          # first query tile staged in K slots 1-2
+    bar("q_full", 1); bar("qstage_free", 8)          # each segment's query staged in K slots 1-2
     bar("xchg", 2)                                   # one quadrant's two warps, one per half
     for i in range(n_rec):
         bar(f"p_full{i}", 4)                         # the four warps of the writing half
@@ -77,14 +77,18 @@ def roles(segs, rescale, k_slots, n_rec):
     def score_tma():
         fit = 0
         for seg, (lo, hi) in enumerate(segs):
-            if seg == 0:
-                B["q_full"].arrive()                 # the first query tile's bytes land
+            if fit > 0:                              # the ring drained: the last fill consumed
+                k = fit - 1
+                yield wait(f"k_empty{k % k_slots}", (k // k_slots) & 1, k // k_slots)
+            B["q_full"].arrive()                     # the segment's query tile lands in slots 1-2
+            staged = True
             for _j, _nb in _passes(lo, hi):
                 for _f in range(FILLS):
                     s = fit % k_slots
                     yield wait(f"k_empty{s}", ((fit // k_slots) & 1) ^ 1, fit // k_slots - 1)
-                    if fit == 1:                     # slots 1-2 free once the tile moved to TMEM
-                        yield wait("qstage_free", 0, 0)
+                    if staged and s != 0:            # slots 1-2 free once the tile moved to TMEM
+                        yield wait("qstage_free", seg & 1, seg)
+                        staged = False
                     B[f"k_full{s}"].arrive()
                     fit += 1
 
@@ -108,9 +112,8 @@ def roles(segs, rescale, k_slots, n_rec):
         for seg, (lo, hi) in enumerate(segs):
             if seg > 0:
                 yield wait("q_free", (seg - 1) & 1, seg - 1)
-            else:
-                yield wait("q_full", 0, 0)
-                B["qstage_free"].arrive(4)           # lane 0 of each of the half's four warps
+            yield wait("q_full", seg & 1, seg)
+            B["qstage_free"].arrive(4)               # lane 0 of each of the half's four warps
             B["q_ready"].arrive(128)
             for j0, nb in _passes(lo, hi):
                 yield wait("s_full", pit & 1, pit)
