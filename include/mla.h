@@ -29,8 +29,15 @@
  *     multiple of 16 in [16, 128].
  *   - bf16 = IEEE binary32 upper half; fp8 = OCP E4M3 (bias 7, max 448, NaN
  *     S.1111.111, no infinities).  Outputs are rounded to nearest even.
- *   - Thread safety: stateless; concurrent calls on different streams are safe
- *     provided they use different output and workspace buffers.
+ *   - State kept by the library: the wait bound of mla_set_wait_limit
+ *     (process-wide), the MLA_SPLITS value (read once per process), per-device
+ *     kernel attributes set on first use, the text of each host thread's last
+ *     CUDA error (mla_last_error_string) and mla_decode_noalloc's scratch
+ *     array (shared by every call on a device).  No other call keeps state
+ *     between calls: the caller's workspace carries each decode's scratch and
+ *     error word.  Concurrent calls on different streams are safe provided
+ *     they use different output and workspace buffers (and, for
+ *     mla_decode_noalloc, do not overlap on one device).
  */
 #ifndef MLA_H_
 #define MLA_H_

@@ -49,6 +49,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "schedule.cuh"
@@ -959,15 +961,15 @@ size_t decode_sm100_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_decode_sm100(const DecodeParams& p, const CUtensorMap& tmap, const CUtensorMap& qmap,
                                 cudaStream_t stream) {
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(kSmemBytes));
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * p.P);
