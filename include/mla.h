@@ -55,7 +55,8 @@ typedef enum {
     MLA_ERR_UNSUPPORTED = 2,         /* valid request this build does not handle */
     MLA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < mla_decode_workspace_bytes(...) */
     MLA_ERR_CUDA = 4,                /* a CUDA runtime/driver call or launch failed */
-    MLA_ERR_DEVICE = 5               /* device-side error bits were set (mla_get_device_error) */
+    MLA_ERR_DEVICE = 5               /* reserved, returned by no call: device-side problems are
+                                        MLA_DEVERR_* bits read by the *_get_error calls */
 } mla_status_t;
 
 typedef enum {
