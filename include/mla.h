@@ -102,7 +102,9 @@ mla_status_t mla_absorb_o(const void *o_latent, const void *w_uv, void *out, int
  * mla_absorb_get_error - device error bits of the mla_absorb_q / mla_absorb_o launches since
  * the last call (MLA_DEVERR_TIMEOUT when a bounded wait in the kernel gave up;
  * the affected rows are then not written).  Synchronises `stream` and clears
- * the bits.  MLA_ERR_INVALID_ARG if err_bits is NULL.
+ * the bits.  The error word is one per device and process: absorption calls on
+ * different streams (or threads) record into, and this call clears, the same
+ * word.  MLA_ERR_INVALID_ARG if err_bits is NULL.
  */
 mla_status_t mla_absorb_get_error(void *stream, uint32_t *err_bits);
 
@@ -309,7 +311,9 @@ mla_status_t mla_cache_quantize_fp8(const void *cache_bf16, const int32_t *block
 
 /*
  * mla_cache_get_error - device error bits of the cache writers since the last
- * call; synchronises `stream` and clears them.
+ * call; synchronises `stream` and clears them.  As for the absorption, the
+ * word is one per device and process, shared by calls on every stream.
+ * MLA_ERR_INVALID_ARG if err_bits is NULL.
  */
 mla_status_t mla_cache_get_error(void *stream, uint32_t *err_bits);
 
@@ -319,7 +323,8 @@ mla_status_t mla_cache_get_error(void *stream, uint32_t *err_bits);
  * seconds of SM clock; cycles <= 0 restores the default).  Returns the
  * previous bound.  A wait that reaches the bound records MLA_DEVERR_TIMEOUT,
  * makes every role of the kernel leave its loop, lets copies in flight land
- * and exits; the outputs of that launch are then undefined, the context stays
+ * and exits; the outputs of that launch are then undefined (mla_decode writes
+ * them as out = 0, lse = NaN while the bit is set), the context stays
  * usable.  Meant for tests of that failure path and for diagnosis.
  */
 long long mla_set_wait_limit(long long cycles);
