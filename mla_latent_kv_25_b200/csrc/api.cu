@@ -10,6 +10,7 @@
 #include "../../include/mla.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "plan.h"
 
 namespace {
 
@@ -144,25 +145,6 @@ constexpr int kMaxTiledRows = 8 * kMaxHeads;
 
 bool valid_rows(int rows) {
   return valid_heads(rows) || (rows > kMaxHeads && rows <= kMaxTiledRows && rows % kMaxHeads == 0);
-}
-
-// The fp8 cache's widened bf16 copy, placed after the split-KV workspace:
-// a scratch block table int32 [B * max_blocks] and a dense bf16 cache
-// [B * max_blocks, 64, 576] (block b * max_blocks + j holds logical block j
-// of sequence b).  Its block ids and TMA row coordinates must fit int32.
-constexpr long long kMaxWideBlocks = 1LL << 24;
-
-struct WideLayout {
-  size_t table, cache, total;
-};
-
-WideLayout wide_layout(size_t split_ws_total, int B, int max_blocks) {
-  const size_t n = size_t(B) * size_t(max_blocks);
-  WideLayout w;
-  w.table = align256(split_ws_total);
-  w.cache = align256(w.table + n * 4);
-  w.total = w.cache + n * kBlock * kRow * 2;
-  return w;
 }
 
 }  // namespace
@@ -401,21 +383,10 @@ mla_status_t decode_rows(const void* q, int q_len, mla_cache_dtype_t cache_dtype
   // workspace, then decoded like a bf16 cache.  One group when the workspace
   // holds the whole batch's widened copy (mla_decode_fp8_workspace_bytes);
   // else the largest groups (and, if need be, fewer split-KV engines) that fit.
-  int Bg = B, Pg = P;
-  for (;;) {
-    const long long wide_blocks = static_cast<long long>(Bg) * max_blocks_per_seq;
-    if (wide_blocks <= kMaxWideBlocks &&
-        wide_layout(ws_layout(Bg, rows, Pg).total, Bg, max_blocks_per_seq).total <= workspace_bytes)
-      break;
-    if (Pg > 1) {
-      Pg = (Pg + 1) / 2;
-    } else if (Bg > 1) {
-      Bg = (Bg + 1) / 2;
-      Pg = resolve_engines(num_splits, Bg);
-    } else {
-      return MLA_ERR_WORKSPACE_TOO_SMALL;
-    }
-  }
+  const Fp8Plan plan = plan_fp8_groups(B, rows, max_blocks_per_seq, P, workspace_bytes,
+                                       [&](int n) { return resolve_engines(num_splits, n); });
+  if (plan.Bg == 0) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  const int Bg = plan.Bg, Pg = plan.Pg;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   for (int b0 = 0; b0 < B; b0 += Bg) {
     const int nb = min(Bg, B - b0);

@@ -6,6 +6,7 @@
 #include <vector>
 
 #include "../mla_latent_kv_25_b200/csrc/common.cuh"
+#include "../mla_latent_kv_25_b200/csrc/plan.h"
 
 using namespace mla;
 
@@ -72,6 +73,43 @@ int main() {
     CHECK(w.seq_info >= 4 && w.lse_part >= w.seq_info + size_t(B) * 16, "seq_info overlaps");
     CHECK(w.o_part >= w.lse_part + size_t(2 * P) * H * 4, "lse_part overlaps");
     CHECK(w.total >= w.o_part + size_t(2 * P) * H * kDc * 4, "o_part overflows");
+    ++cases;
+  }
+  // fp8 decode groups (plan.h): every group fits the workspace, the groups
+  // cover the batch, the whole batch at the requested engine count when it
+  // fits, and no plan only when not even one sequence on one engine fits
+  for (int it = 0; it < 4000; ++it) {
+    const int B = 1 + static_cast<int>(next() % 300);
+    const int rows = 16 * (1 + static_cast<int>(next() % 8));
+    const int mb = 1 + static_cast<int>(next() % (it % 4 == 0 ? 4096 : 256));
+    const int cap = 1 + static_cast<int>(next() % 148);
+    auto engines_for = [&](int n) { return n < cap ? n : cap; };
+    const int P = engines_for(B);
+    const size_t whole = fp8_group_bytes(B, rows, mb, P);
+    const size_t one = fp8_group_bytes(1, rows, mb, 1);
+    size_t ws = 0;
+    switch (it % 4) {
+      case 0: ws = whole; break;                                    // exactly the whole batch
+      case 1: ws = one + next() % (whole > one ? whole - one : 1); break;  // between
+      case 2: ws = one > 0 ? one - 1 - next() % (one < 1000 ? one : 1000) : 0; break;  // too small
+      default: ws = static_cast<size_t>(next() % (whole + 1)); break;
+    }
+    const Fp8Plan plan = plan_fp8_groups(B, rows, mb, P, ws, engines_for);
+    if (plan.Bg == 0) {
+      CHECK(one == 0 || one > ws, "no plan although one sequence fits (B=%d mb=%d ws=%zu one=%zu)", B, mb, ws, one);
+      continue;
+    }
+    CHECK(plan.Bg >= 1 && plan.Bg <= B && plan.Pg >= 1, "plan out of range Bg=%d Pg=%d", plan.Bg, plan.Pg);
+    if (whole != 0 && whole <= ws) CHECK(plan.Bg == B && plan.Pg == P, "whole batch fits but Bg=%d Pg=%d", plan.Bg, plan.Pg);
+    int covered = 0;
+    for (int b0 = 0; b0 < B; b0 += plan.Bg) {
+      const int n = B - b0 < plan.Bg ? B - b0 : plan.Bg;
+      const int pg = plan.Pg < engines_for(n) ? plan.Pg : engines_for(n);
+      const size_t need = fp8_group_bytes(n, rows, mb, pg);
+      CHECK(need != 0 && need <= ws, "group at %d (n=%d, %d engines) needs %zu > %zu", b0, n, pg, need, ws);
+      covered += n;
+    }
+    CHECK(covered == B, "groups cover %d of %d", covered, B);
     ++cases;
   }
   std::printf("ok %d\n", cases);
