@@ -99,3 +99,38 @@ def test_noalloc_fp8_cache_matches_decode():
     torch.cuda.synchronize()
     assert_close(to_np(out).reshape(-1, 512), to_np(ref_out).reshape(-1, 512), "noalloc fp8 out")
     assert_close(to_np(lse).reshape(-1), to_np(ref_lse).reshape(-1), "noalloc fp8 lse")
+
+
+@pytest.mark.gpu
+def test_noalloc_timeout_after_a_wide_split_call_stays_defined():
+    """The built-in scratch keeps the previous call's per-sequence records: a
+    call cut over 512 engines (B=1, H=16) leaves records naming high engine
+    slots; a following H=128 call whose waits expire must not merge from
+    them.  Its rows read out = 0, lse = NaN, the timeout bit is reported by
+    mla_decode_noalloc_get_error, and the next call is right again."""
+    w1 = inputs.make("v3", B=1, H=16, L=[5000], seed=49)
+    d1 = binding.to_device(w1)
+    out1 = torch.empty((1, 16, 512), dtype=torch.bfloat16, device="cuda")
+    lse1 = torch.empty((1, 16), dtype=torch.float32, device="cuda")
+    assert _noalloc_raw(d1, w1, out1, lse1, 512) == 0
+    assert binding.mla_decode_noalloc_get_error() == 0
+    w2 = inputs.make("v3", B=2, H=128, L=[3000, 700], seed=50)
+    d2 = binding.to_device(w2)
+    out2 = torch.full((2, 128, 512), 7.0, dtype=torch.bfloat16, device="cuda")
+    lse2 = torch.full((2, 128), 7.0, dtype=torch.float32, device="cuda")
+    prev = binding.mla_set_wait_limit(1000)
+    try:
+        st = _noalloc_raw(d2, w2, out2, lse2, 4)
+        torch.cuda.synchronize()
+    finally:
+        binding.mla_set_wait_limit(0)
+    assert st == 0, binding.STATUS.get(st, st)
+    err = binding.mla_decode_noalloc_get_error()
+    assert err & binding.DEVERR_TIMEOUT and not err & binding.DEVERR_BAD_PIECES
+    assert torch.all(out2 == 0) and torch.all(torch.isnan(lse2))
+    ref_out, ref_lse, ws = binding.decode_device(d2, w2.softmax_scale, num_splits=4)
+    assert _noalloc_raw(d2, w2, out2, lse2, 4) == 0
+    torch.cuda.synchronize()
+    assert binding.mla_decode_noalloc_get_error() == 0
+    assert_close(to_np(out2).reshape(-1, 512), to_np(ref_out).reshape(-1, 512), "noalloc after timeout out")
+    assert_close(to_np(lse2).reshape(-1), to_np(ref_lse).reshape(-1), "noalloc after timeout lse")
