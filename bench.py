@@ -503,27 +503,41 @@ def run_ours(args, world, rank, local):
     if binding.mla_absorb_get_error(stream) != 0:
         raise RuntimeError("device error in the output absorption")
 
-    # multi-token decode, timed on its own: the same query rows regrouped as
-    # 2 tokens x H/2 heads per sequence (drafts causal among themselves)
+    # multi-token decode at the workload's H, timed on its own: q_len draft
+    # tokens of H heads per sequence (token 0 = this step's queries, the
+    # others seeded normal draws with the queries' spread), causal among the drafts;
+    # q_len * H rows above 128 run in 128-row tiles, one cache pass each
     multi = None
-    if H % 32 == 0 and not fp8:
-        q2 = q.view(B, 2, H // 2, 576)
-        out2 = torch.empty((B, 2, H // 2, 512), dtype=torch.bfloat16, device=dev)
-        lse2 = torch.empty((B, 2, H // 2), dtype=torch.float32, device=dev)
-        ws2 = binding.alloc_workspace(B, H, args.num_splits, device=dev)
+    if not fp8 and H == 128:
+        multi = []
+        gen = torch.Generator().manual_seed(1234)
+        for q_len in (2, 4):
+            extra = (torch.randn((B, q_len - 1, H, 576), generator=gen) * float(q.float().std())).to(torch.bfloat16)
+            qm = torch.cat([q.view(B, 1, H, 576), extra.to(dev)], dim=1).contiguous()
+            outm = torch.empty((B, q_len, H, 512), dtype=torch.bfloat16, device=dev)
+            lsem = torch.empty((B, q_len, H), dtype=torch.float32, device=dev)
+            wsm = binding.alloc_workspace(B, q_len * H, args.num_splits, device=dev)
 
-        def mcall():
-            binding.mla_decode_multi(q2, d["cache"], d["block_table"], d["seq_lens"],
-                                     w.softmax_scale, out2, lse2, ws2, num_splits=args.num_splits,
-                                     stream=stream)
-        for _ in range(3):
-            mcall()
-        m_ms = float(np.mean(time_launches(mcall, 100, stream)))
-        if binding.mla_get_device_error(ws2, stream) != 0:
-            raise RuntimeError("device error in the multi-token decode")
-        multi = {"q_len": 2, "heads_per_token": H // 2, "rows_per_sequence": H,
-                 "note": "the same query rows regrouped as 2 draft tokens x H/2 heads",
-                 "ms_per_launch": round(m_ms, 5)}
+            def mcall(qm=qm, outm=outm, lsem=lsem, wsm=wsm):
+                binding.mla_decode_multi(qm, d["cache"], d["block_table"], d["seq_lens"],
+                                         w.softmax_scale, outm, lsem, wsm, num_splits=args.num_splits,
+                                         stream=stream)
+            for _ in range(3):
+                mcall()
+            m_ms = float(np.mean(time_launches(mcall, 50, stream)))
+            if binding.mla_get_device_error(wsm, stream) != 0:
+                raise RuntimeError("device error in the multi-token decode")
+            mb = layout.decode_algorithmic_bytes(w.total_tokens, B, q_len * H, "bf16")
+            mf = layout.decode_flops(w.total_tokens, q_len * H)
+            t_hbm = mb / (float(peaks["hbm_gbs"]) * 1e9) * 1e3
+            t_tc = mf / (float(peaks["bf16_tflops"]) * 1e12) * 1e3
+            multi.append({"q_len": q_len, "heads_per_token": H, "rows_per_sequence": q_len * H,
+                          "cache_passes": (q_len * H + 127) // 128,
+                          "ms_per_launch": round(m_ms, 5), "algorithmic_bytes": mb, "flops": mf,
+                          "bound": "tensor" if t_tc > t_hbm else "hbm",
+                          "roofline_ms": round(max(t_hbm, t_tc), 5),
+                          "frac": round(max(t_hbm, t_tc) / m_ms, 4)})
+            del qm, outm, lsem, wsm
     if binding.mla_get_device_error(ws, stream) != 0:
         raise RuntimeError("device error during timing")
 
@@ -576,9 +590,7 @@ def run_ours(args, world, rank, local):
                     "pipelined": "double-buffered; copies on their own streams overlap compute"},
             "gpu_launches": launches_per_step * K,
             "absorb_o": absorb_o_line(B, H, absorb_o_ms, float(peaks["hbm_gbs"])),
-            "multi_token": None if multi is None else dict(
-                multi, algorithmic_bytes=dec_b,
-                frac=round(dec_b / (multi["ms_per_launch"] * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4)),
+            "multi_token": multi,
             "workloads": extras or None,
             "clocks": clk,
         }
