@@ -281,3 +281,25 @@ def test_model_finds_a_planted_deadlock():
     finally:
         Bar.__init__ = orig
     assert all(b is not True for b in blocked)
+
+
+def _with_planted_count(name_prefix, count):
+    orig = Bar.__init__
+
+    def planted(self, name, c):
+        orig(self, name, count if name.startswith(name_prefix) else c)
+    return orig, planted
+
+
+def test_model_finds_a_planted_query_staging_fault():
+    """Planted fault: the query-staging release expects nine warp arrivals
+    where the eight softmax warps give eight: the TMA warp then never refills
+    K slots 1-2 and the pipeline stops, on the first segment and on later
+    ones."""
+    orig, planted = _with_planted_count("qstage_free", 9)
+    Bar.__init__ = planted
+    try:
+        blocked = [simulate(segs, seed) for segs in ([(0, 9)], [(0, 3), (3, 11)]) for seed in range(3)]
+    finally:
+        Bar.__init__ = orig
+    assert all(b is not True for b in blocked)
